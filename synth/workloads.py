@@ -1,0 +1,241 @@
+"""Seeded synthetic workloads (shapes, value distributions, sinks, page tables, planted mappings).
+
+Every array is drawn from ``numpy.random.default_rng(seed)`` (PCG64) in float32 in a fixed draw
+order, then rounded to bf16 with round-to-nearest-even. bf16 tensors are carried as ``uint16``
+bit patterns so that both the oracle (which upcasts them exactly to float64) and the CUDA path
+(which views them as ``torch.bfloat16``) see the same numbers.
+
+Workloads (one per configuration of the benchmark description):
+
+* ``tiny``       n=512, H_s=8, d=64, H_r=4, d_v=64, B=64, tau=0.95, std 1.5, sink, seed 0
+* ``prefill8k``  n=8192, H_s=32, d=128, H_r=24, d_v=128, tau=0.95, std 1.5, sink,
+                 local bias +2.0 on |i-j| < 128
+* ``varlen40k``  4 packed sequences 4096/8192/12288/16384 (40960 tokens), H_s=40, H_r=32,
+                 d=d_v=128, tau=0.9, std 1.5, sink on token 0 of every sequence
+* head match     n=1024, small 24 layers x 14 heads d=64, large 8 layers x 64 heads d=128,
+                 each large head a noisy zero-padded copy of a uniformly drawn small head
+* decode         batch 4, context 8704, sender 14 heads, receiver 64 heads d_v=128, one-hot
+                 W, V cache in 16-token pages under a random page table
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------------------------
+# bf16 bit handling (rounding of random draws; not part of the method)
+# ----------------------------------------------------------------------------------------------
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (round-to-nearest-even); return the uint16 bit patterns."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    nan = np.isnan(x)
+    if nan.any():
+        r[nan] = 0x7FC0
+    return r
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Exact upcast of bf16 bit patterns to float32."""
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    """Exact upcast of bf16 bit patterns to float64."""
+    return bf16_bits_to_f32(b).astype(np.float64)
+
+
+def _normal_bits(rng: np.random.Generator, shape, std: float) -> np.ndarray:
+    x = rng.standard_normal(shape, dtype=np.float32)
+    if std != 1.0:
+        x *= np.float32(std)
+    return x
+
+
+# ----------------------------------------------------------------------------------------------
+# Prefill workloads: map_compress + mapped_av
+# ----------------------------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class PrefillWorkload:
+    name: str
+    seqlens: list
+    H_s: int
+    d: int
+    H_r: int
+    d_v: int
+    B: int
+    tau: float
+    bias_window: int
+    bias_value: float
+    q: np.ndarray          # uint16 bf16 bits [n, H_s, d]
+    k: np.ndarray          # uint16 bf16 bits [n, H_s, d]
+    v: np.ndarray          # uint16 bf16 bits [n, H_r, d_v]
+    W: np.ndarray          # float32 [H_r, H_s]
+    cu_seqlens: np.ndarray  # int32 [S+1]
+
+    @property
+    def n(self) -> int:
+        return int(self.cu_seqlens[-1])
+
+    @property
+    def num_seqs(self) -> int:
+        return len(self.seqlens)
+
+
+PREFILL_CONFIGS = {
+    "tiny": dict(seqlens=[512], H_s=8, d=64, H_r=4, d_v=64, B=64, tau=0.95, std=1.5,
+                 sink=True, bias_window=0, bias_value=0.0),
+    "prefill8k": dict(seqlens=[8192], H_s=32, d=128, H_r=24, d_v=128, B=64, tau=0.95, std=1.5,
+                      sink=True, bias_window=128, bias_value=2.0),
+    "varlen40k": dict(seqlens=[4096, 8192, 12288, 16384], H_s=40, d=128, H_r=32, d_v=128, B=64,
+                      tau=0.9, std=1.5, sink=True, bias_window=0, bias_value=0.0),
+}
+
+
+def make_prefill(seqlens, H_s, d, H_r, d_v, B=64, tau=0.95, std=1.5, sink=True,
+                 bias_window=0, bias_value=0.0, seed=0, name="custom",
+                 q_zero=False, v_const=None) -> PrefillWorkload:
+    """Draw Q, K, V (bf16) and W (fp32) in the order Q, K, V, W.
+
+    ``sink`` multiplies the key of token 0 of every sequence by 4 (a power of two, so exact) before
+    bf16 rounding. ``q_zero`` zeroes Q (uniform attention rows); ``v_const`` replaces V by that
+    constant. Both are for closed-form checks.
+    """
+    seqlens = [int(x) for x in seqlens]
+    n = int(sum(seqlens))
+    cu = np.zeros(len(seqlens) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(seqlens)
+    rng = np.random.default_rng(seed)
+    q = _normal_bits(rng, (n, H_s, d), std)
+    k = _normal_bits(rng, (n, H_s, d), std)
+    v = _normal_bits(rng, (n, H_r, d_v), std)
+    W = rng.standard_normal((H_r, H_s), dtype=np.float32) * np.float32(math.sqrt(1.0 / H_s))
+    if sink:
+        for s in range(len(seqlens)):
+            if seqlens[s] > 0:
+                k[cu[s]] *= np.float32(4.0)
+    if q_zero:
+        q[:] = 0.0
+    if v_const is not None:
+        v[:] = np.float32(v_const)
+    return PrefillWorkload(name=name, seqlens=seqlens, H_s=H_s, d=d, H_r=H_r, d_v=d_v, B=B,
+                           tau=float(tau), bias_window=int(bias_window),
+                           bias_value=float(bias_value), q=bf16_bits(q), k=bf16_bits(k),
+                           v=bf16_bits(v), W=np.ascontiguousarray(W, dtype=np.float32),
+                           cu_seqlens=cu)
+
+
+def prefill_config(name: str, seed: int = 0) -> PrefillWorkload:
+    c = dict(PREFILL_CONFIGS[name])
+    return make_prefill(seed=seed, name=name, **c)
+
+
+# ----------------------------------------------------------------------------------------------
+# Head-match calibration workload
+# ----------------------------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class HeadMatchWorkload:
+    n: int
+    L_s: int
+    H_small: int
+    d_small: int
+    L_l: int
+    H_large: int
+    d_large: int
+    q_small: np.ndarray   # uint16 bf16 [L_s, n, H_small, d_small]
+    k_small: np.ndarray
+    q_large: np.ndarray   # uint16 bf16 [L_l, n, H_large, d_large]
+    k_large: np.ndarray
+    planted: np.ndarray   # int32 [L_l, H_large]: small head index (layer * H_small + head)
+
+
+def make_head_match(n=1024, L_s=24, H_small=14, d_small=64, L_l=8, H_large=64, d_large=128,
+                    noise=0.3, seed=0) -> HeadMatchWorkload:
+    """Small Q, K ~ N(0,1); each large head copies a uniformly drawn small head's Q and K into
+    dims [0, d_small), zero elsewhere, plus N(0, noise^2) on every dim. Draw order: small Q,
+    small K, planted assignment, large-Q noise, large-K noise."""
+    rng = np.random.default_rng(seed)
+    qs = rng.standard_normal((L_s, n, H_small, d_small), dtype=np.float32)
+    ks = rng.standard_normal((L_s, n, H_small, d_small), dtype=np.float32)
+    planted = rng.integers(0, L_s * H_small, size=(L_l, H_large)).astype(np.int32)
+    nq = rng.standard_normal((L_l, n, H_large, d_large), dtype=np.float32) * np.float32(noise)
+    nk = rng.standard_normal((L_l, n, H_large, d_large), dtype=np.float32) * np.float32(noise)
+    ql = nq
+    kl = nk
+    dd = min(d_small, d_large)
+    for ll in range(L_l):
+        for h in range(H_large):
+            s = int(planted[ll, h])
+            ql[ll, :, h, :dd] += qs[s // H_small, :, s % H_small, :dd]
+            kl[ll, :, h, :dd] += ks[s // H_small, :, s % H_small, :dd]
+    return HeadMatchWorkload(n=n, L_s=L_s, H_small=H_small, d_small=d_small, L_l=L_l,
+                             H_large=H_large, d_large=d_large, q_small=bf16_bits(qs),
+                             k_small=bf16_bits(ks), q_large=bf16_bits(ql), k_large=bf16_bits(kl),
+                             planted=planted)
+
+
+def head_match_config(seed: int = 0) -> HeadMatchWorkload:
+    return make_head_match(seed=seed)
+
+
+# ----------------------------------------------------------------------------------------------
+# Decode workload (paged V cache, one-hot W)
+# ----------------------------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class DecodeWorkload:
+    batch: int
+    ctx_lens: np.ndarray    # int32 [batch]
+    H_s: int
+    H_r: int
+    d_v: int
+    page_size: int
+    p_rows: np.ndarray      # float32 [batch, H_s, max_ctx]; each row a probability vector
+    W: np.ndarray           # float32 [H_r, H_s] (one-hot rows)
+    assign: np.ndarray      # int32 [H_r]: the sender head of each receiver head
+    v_pages: np.ndarray     # uint16 bf16 [num_pages, page_size, H_r, d_v]
+    page_table: np.ndarray  # int32 [batch, max_pages]
+
+
+def make_decode(batch=4, ctx=8704, H_s=14, H_r=64, d_v=128, page_size=16, sink_weight=64.0,
+                ctx_lens=None, seed=0) -> DecodeWorkload:
+    """Draw order: sender rows, one-hot assignment, V pages, page-table permutation.
+
+    The sender's attention rows are drawn from a Dirichlet distribution (normalised Gamma draws)
+    with a heavier concentration at position 0, a stand-in for a causal softmax row with a sink.
+    Unused tail positions (ctx_len < max) are zero.
+    """
+    if ctx_lens is None:
+        ctx_lens = [ctx] * batch
+    ctx_lens = np.asarray(ctx_lens, dtype=np.int32)
+    max_ctx = int(ctx_lens.max())
+    max_pages = (max_ctx + page_size - 1) // page_size
+    rng = np.random.default_rng(seed)
+    g = rng.gamma(shape=1.0, scale=1.0, size=(batch, H_s, max_ctx))
+    g[:, :, 0] *= sink_weight
+    for b in range(batch):
+        g[b, :, ctx_lens[b]:] = 0.0
+    p_rows = (g / g.sum(axis=2, keepdims=True)).astype(np.float32)
+    assign = rng.integers(0, H_s, size=H_r).astype(np.int32)
+    W = np.zeros((H_r, H_s), dtype=np.float32)
+    W[np.arange(H_r), assign] = 1.0
+    num_pages = batch * max_pages
+    v = rng.standard_normal((num_pages, page_size, H_r, d_v), dtype=np.float32)
+    perm = rng.permutation(num_pages).astype(np.int32)
+    page_table = perm.reshape(batch, max_pages)
+    return DecodeWorkload(batch=batch, ctx_lens=ctx_lens, H_s=H_s, H_r=H_r, d_v=d_v,
+                          page_size=page_size, p_rows=p_rows, W=W, assign=assign,
+                          v_pages=bf16_bits(v), page_table=page_table)
+
+
+def decode_config(seed: int = 0) -> DecodeWorkload:
+    return make_decode(seed=seed)
