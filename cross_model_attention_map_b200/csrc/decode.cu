@@ -1,0 +1,181 @@
+// mapped_av_paged: the decode step of a mapped layer. The large model's mapped layer reuses the
+// small model's attention row directly (no Q/K projection, no QK^T, no K cache) and only streams
+// its own V cache ("IAM: Efficient Inference through Attention Mapping between Different-scale
+// LLMs" notes, Method section 4, decode bullet); with a general W the row is the linear
+// combination of sender heads used by mapped_av.
+//
+//   out[b, r, :] = sum_{j < ctx[b]} (sum_s W[r, s] p[b, s, j]) V[page(b, j), j % page, r, :]
+//
+// The V cache stream dominates (bytes read once), so the kernel is a coalesced GEMV on CUDA
+// cores: CTA (chunk of pages, sequence b, slice of 8192 output elements) walks its pages; each
+// thread owns four 16-byte chunks of the [H_r * d_v] token row and accumulates fp32. The mixed
+// weights of the page's tokens are formed in shared memory first. Partial sums per page chunk go
+// to the workspace and a second kernel adds them in a fixed order (deterministic).
+#include "internal.h"
+
+namespace iamap {
+
+constexpr int kDecThreads = 256;
+constexpr int kDecCPT = 4;                                  // 16-byte chunks per thread
+constexpr int kDecSlice = kDecThreads * kDecCPT * 8;        // output elements per CTA slice
+constexpr int kDecMaxPage = 32;                             // largest page size supported
+constexpr int kDecMaxH = 128;                               // largest H_s / H_r supported
+
+struct DecParams {
+  const float* p_rows;
+  int ctx_stride;
+  const float* W;
+  const __nv_bfloat16* v;
+  int64_t num_pages;
+  const int32_t* page_table;
+  int max_pages;
+  int page_size;
+  const int32_t* ctx_lens;
+  int H_s, H_r, d_v;
+  int chunks, ppc;
+  float* partial;
+  unsigned int* status;
+};
+
+__global__ void __launch_bounds__(kDecThreads) paged_gemv_kernel(DecParams p) {
+  __shared__ float s_p[kDecMaxPage * kDecMaxH];    // [slot][s] sender probabilities
+  __shared__ float s_w[kDecMaxPage * kDecMaxH];    // [slot][r] mixed weights
+  const int chunk = blockIdx.x, b = blockIdx.y, slice = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int E = p.H_r * p.d_v;
+  const int ctx = p.ctx_lens[b];
+  const int npages = (ctx + p.page_size - 1) / p.page_size;
+  const int pg0 = chunk * p.ppc, pg1 = min(npages, pg0 + p.ppc);
+  const int e0 = slice * kDecSlice;
+
+  float acc[kDecCPT][8];
+#pragma unroll
+  for (int c = 0; c < kDecCPT; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[c][e] = 0.f;
+  int head_of[kDecCPT];
+  bool live[kDecCPT];
+#pragma unroll
+  for (int c = 0; c < kDecCPT; ++c) {
+    const int e = e0 + (c * kDecThreads + tid) * 8;
+    live[c] = e < E;
+    head_of[c] = live[c] ? e / p.d_v : 0;
+  }
+  const float* prow = p.p_rows + (int64_t)b * p.H_s * p.ctx_stride;
+  bool bad = false;
+  for (int pi = pg0; pi < pg1; ++pi) {
+    const int j0 = pi * p.page_size;
+    const int nslot = min(p.page_size, ctx - j0);
+    __syncthreads();
+    for (int e = tid; e < p.page_size * p.H_s; e += kDecThreads) {
+      const int t = e / p.H_s, sh = e % p.H_s;
+      s_p[t * kDecMaxH + sh] = t < nslot ? prow[(int64_t)sh * p.ctx_stride + j0 + t] : 0.f;
+    }
+    __syncthreads();
+    for (int e = tid; e < p.page_size * p.H_r; e += kDecThreads) {
+      const int t = e / p.H_r, r = e % p.H_r;
+      float w = 0.f;
+      for (int sh = 0; sh < p.H_s; ++sh) w = fmaf(p.W[r * p.H_s + sh], s_p[t * kDecMaxH + sh], w);
+      s_w[t * kDecMaxH + r] = w;
+    }
+    __syncthreads();
+    const int pg = p.page_table[(int64_t)b * p.max_pages + pi];
+    if (pg < 0 || pg >= p.num_pages) {
+      bad = true;
+      continue;
+    }
+    const __nv_bfloat16* vpage = p.v + (int64_t)pg * p.page_size * E;
+    for (int t = 0; t < nslot; ++t) {
+      uint4 raw[kDecCPT];
+#pragma unroll
+      for (int c = 0; c < kDecCPT; ++c)
+        if (live[c])
+          raw[c] = __ldg(reinterpret_cast<const uint4*>(vpage + (int64_t)t * E + e0 +
+                                                        (c * kDecThreads + tid) * 8));
+#pragma unroll
+      for (int c = 0; c < kDecCPT; ++c) {
+        if (!live[c]) continue;
+        const float w = s_w[t * kDecMaxH + head_of[c]];
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[c]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+          acc[c][2 * e] = fmaf(w, f.x, acc[c][2 * e]);
+          acc[c][2 * e + 1] = fmaf(w, f.y, acc[c][2 * e + 1]);
+        }
+      }
+    }
+  }
+  if (bad) raise_status(p.status, IAMAP_DEV_BAD_INDEX);
+  float* dst = p.partial + ((int64_t)b * p.chunks + chunk) * E + e0;
+#pragma unroll
+  for (int c = 0; c < kDecCPT; ++c) {
+    if (!live[c]) continue;
+    float4* d4 = reinterpret_cast<float4*>(dst + (c * kDecThreads + tid) * 8);
+    d4[0] = make_float4(acc[c][0], acc[c][1], acc[c][2], acc[c][3]);
+    d4[1] = make_float4(acc[c][4], acc[c][5], acc[c][6], acc[c][7]);
+  }
+}
+
+__global__ void paged_reduce_kernel(const float* __restrict__ partial, int chunks, int E,
+                                    float* __restrict__ out) {
+  const int b = blockIdx.y;
+  const int e = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (e >= E) return;
+  const float* src = partial + (int64_t)b * chunks * E + e;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = 0; c < chunks; ++c) {
+    const float4 x = *reinterpret_cast<const float4*>(src + (int64_t)c * E);
+    acc.x += x.x;
+    acc.y += x.y;
+    acc.z += x.z;
+    acc.w += x.w;
+  }
+  *reinterpret_cast<float4*>(out + (int64_t)b * E + e) = acc;
+}
+
+void paged_split(int batch, int max_ctx, int page_size, int num_sms, int* chunks,
+                 int* pages_per_chunk) {
+  const int npages = (max_ctx + page_size - 1) / page_size;
+  int want = (2 * num_sms + batch - 1) / batch;
+  if (want < 1) want = 1;
+  int ppc = (npages + want - 1) / want;
+  if (ppc < 1) ppc = 1;
+  int ch = (npages + ppc - 1) / ppc;
+  if (ch < 1) ch = 1;
+  *chunks = ch;
+  *pages_per_chunk = ppc;
+}
+
+int mapped_av_paged_impl(const PagedArgs& a, cudaStream_t stream) {
+  if (a.page_size > kDecMaxPage || a.H_s > kDecMaxH || a.H_r > kDecMaxH)
+    return set_error(IAMAP_ERR_UNSUPPORTED, "page_size <= %d and H_s, H_r <= %d required",
+                     kDecMaxPage, kDecMaxH);
+  DecParams p{};
+  p.p_rows = a.p_rows;
+  p.ctx_stride = a.ctx_stride;
+  p.W = a.W;
+  p.v = static_cast<const __nv_bfloat16*>(a.v_pages);
+  p.num_pages = a.num_pages;
+  p.page_table = a.page_table;
+  p.max_pages = a.max_pages;
+  p.page_size = a.page_size;
+  p.ctx_lens = a.ctx_lens;
+  p.H_s = a.H_s;
+  p.H_r = a.H_r;
+  p.d_v = a.d_v;
+  p.chunks = a.chunks;
+  p.ppc = a.pages_per_chunk;
+  p.partial = a.partial;
+  p.status = a.status;
+  const int E = a.H_r * a.d_v;
+  dim3 grid(a.chunks, a.batch, (E + kDecSlice - 1) / kDecSlice);
+  paged_gemv_kernel<<<grid, kDecThreads, 0, stream>>>(p);
+  IAMAP_LAUNCH_CHECK("paged_gemv_kernel");
+  dim3 rgrid((E / 4 + 255) / 256, a.batch);
+  paged_reduce_kernel<<<rgrid, 256, 0, stream>>>(a.partial, a.chunks, E, a.out);
+  IAMAP_LAUNCH_CHECK("paged_reduce_kernel");
+  return IAMAP_OK;
+}
+
+}  // namespace iamap

@@ -1,0 +1,106 @@
+// Internal launch interfaces between the C ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include "common.cuh"
+
+namespace iamap {
+
+struct CompressArgs {
+  const void* q = nullptr;
+  const void* k = nullptr;
+  const int32_t* cu_seqlens = nullptr;
+  int num_seqs = 0;
+  int64_t n = 0;
+  int H_s = 0, d = 0;
+  float tau = 1.f;
+  int bias_window = 0;
+  float bias_value = 0.f;
+  Plan plan;
+  SeqTables tab;
+  // stage 1 outputs
+  float* lse = nullptr;
+  float* mass = nullptr;
+  uint64_t* headmask_dense = nullptr;
+  int32_t* row_ptr = nullptr;
+  int32_t* col_idx = nullptr;
+  uint64_t* headmask = nullptr;
+  int64_t* val_off = nullptr;
+  int64_t* counts = nullptr;
+  // stage 2 inputs / outputs
+  const float* lse_in = nullptr;
+  const int32_t* row_ptr_in = nullptr;
+  const int32_t* col_idx_in = nullptr;
+  const uint64_t* headmask_in = nullptr;
+  const int64_t* val_off_in = nullptr;
+  const int64_t* counts_in = nullptr;
+  void* vals = nullptr;
+  int64_t capacity = 0;
+  unsigned int* status = nullptr;
+};
+
+int compress_stats_impl(const CompressArgs& a, cudaStream_t stream);
+int compress_extract_impl(const CompressArgs& a, cudaStream_t stream);
+size_t compress_stats_smem(int d, int max_nb);
+size_t compress_extract_smem(int d, int max_nb);
+
+struct MappedAvArgs {
+  const int32_t* cu_seqlens = nullptr;
+  int num_seqs = 0;
+  int64_t n = 0;
+  int H_s = 0;
+  Plan plan;
+  SeqTables tab;
+  const int32_t* row_ptr = nullptr;
+  const int32_t* col_idx = nullptr;
+  const uint64_t* headmask = nullptr;
+  const int64_t* val_off = nullptr;
+  const void* vals = nullptr;
+  int64_t capacity = 0;
+  const float* W = nullptr;
+  int H_r = 0;
+  const void* v = nullptr;
+  int d_v = 0;
+  float* out = nullptr;
+  unsigned int* status = nullptr;
+};
+int mapped_av_impl(const MappedAvArgs& a, cudaStream_t stream);
+
+struct PagedArgs {
+  const float* p_rows = nullptr;
+  int ctx_stride = 0;
+  const float* W = nullptr;
+  const void* v_pages = nullptr;
+  int64_t num_pages = 0;
+  const int32_t* page_table = nullptr;
+  int max_pages = 0;
+  int page_size = 0;
+  const int32_t* ctx_lens = nullptr;
+  int max_ctx = 0;
+  int batch = 0, H_s = 0, H_r = 0, d_v = 0;
+  float* out = nullptr;
+  float* partial = nullptr;  // [batch][chunks][H_r][d_v]
+  int chunks = 0;            // chunks per sequence
+  int pages_per_chunk = 0;
+  unsigned int* status = nullptr;
+};
+void paged_split(int batch, int max_ctx, int page_size, int num_sms, int* chunks,
+                 int* pages_per_chunk);
+int mapped_av_paged_impl(const PagedArgs& a, cudaStream_t stream);
+
+struct HeadMatchArgs {
+  const void* q_small = nullptr;
+  const void* k_small = nullptr;
+  int L_s = 0, H_small = 0, d_small = 0;
+  const void* q_large = nullptr;
+  const void* k_large = nullptr;
+  int L_l = 0, H_large = 0, d_large = 0;
+  int n = 0, n_used = 0;
+  int32_t* argmax = nullptr;
+  float* sim = nullptr;
+  void* ws = nullptr;
+  unsigned int* status = nullptr;
+};
+size_t head_match_ws_bytes(int L_s, int H_small, int L_l, int H_large, int n_used);
+int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream);
+
+}  // namespace iamap

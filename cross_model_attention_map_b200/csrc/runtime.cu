@@ -1,0 +1,183 @@
+// Host plumbing of libiamap: error messages, the per-device context, sequence planning and the
+// device-side scheduling tables shared by the compress and mapped_av kernels.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+namespace iamap {
+
+static thread_local char g_last_error[512] = "";
+
+int set_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+void clear_error() { g_last_error[0] = 0; }
+
+static std::mutex g_ctx_mutex;
+static std::vector<DeviceContext> g_ctx;
+
+DeviceContext* device_context() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    set_error(IAMAP_ERR_CUDA, "cudaGetDevice failed");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_ctx_mutex);
+  if ((int)g_ctx.size() <= dev) g_ctx.resize(dev + 1);
+  DeviceContext& c = g_ctx[dev];
+  if (c.status == nullptr) {
+    unsigned int* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, sizeof(unsigned int));
+    if (e != cudaSuccess) {
+      set_error(IAMAP_ERR_CUDA, "status word allocation failed: %s", cudaGetErrorString(e));
+      return nullptr;
+    }
+    e = cudaMemset(p, 0, sizeof(unsigned int));
+    if (e != cudaSuccess) {
+      cudaFree(p);
+      set_error(IAMAP_ERR_CUDA, "status word init failed: %s", cudaGetErrorString(e));
+      return nullptr;
+    }
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    c.device = dev;
+    c.status = p;
+    c.num_sms = sms;
+  }
+  return &c;
+}
+
+int make_plan(const int32_t* cu_host, int num_seqs, int B, int64_t n, Plan* out) {
+  if (!cu_host) return set_error(IAMAP_ERR_INVALID_ARG, "cu_seqlens_host is null");
+  if (num_seqs < 1) return set_error(IAMAP_ERR_INVALID_ARG, "num_seqs must be >= 1");
+  if (B < 1) return set_error(IAMAP_ERR_INVALID_ARG, "block size must be >= 1");
+  if (cu_host[0] != 0) return set_error(IAMAP_ERR_INVALID_ARG, "cu_seqlens[0] must be 0");
+  Plan p;
+  for (int s = 0; s < num_seqs; ++s) {
+    int64_t L = (int64_t)cu_host[s + 1] - cu_host[s];
+    if (L < 0) return set_error(IAMAP_ERR_INVALID_ARG, "cu_seqlens decreases at %d", s);
+    int64_t nb = (L + B - 1) / B;
+    p.num_rowblocks += nb;
+    p.num_causal_blocks += nb * (nb + 1) / 2;
+    if (nb > p.max_nb) p.max_nb = (int32_t)nb;
+  }
+  if (n >= 0 && (int64_t)cu_host[num_seqs] != n)
+    return set_error(IAMAP_ERR_INVALID_ARG, "cu_seqlens[num_seqs]=%d does not equal n=%lld",
+                     cu_host[num_seqs], (long long)n);
+  if (p.num_causal_blocks >= (int64_t)INT32_MAX)
+    return set_error(IAMAP_ERR_UNSUPPORTED, "more than 2^31 causal blocks");
+  *out = p;
+  return IAMAP_OK;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t seq_tables_bytes(int num_seqs, int64_t num_rowblocks) {
+  return align256(sizeof(int32_t) * (size_t)num_seqs) +
+         2 * align256(sizeof(int32_t) * (size_t)(num_seqs + 1)) +
+         align256(sizeof(int2) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1)) +
+         align256(sizeof(int64_t) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1));
+}
+
+SeqTables carve_seq_tables(void* ws, int num_seqs, int64_t num_rowblocks) {
+  char* p = static_cast<char*>(ws);
+  SeqTables t;
+  t.nb = reinterpret_cast<int32_t*>(p);
+  p += align256(sizeof(int32_t) * (size_t)num_seqs);
+  t.rb_start = reinterpret_cast<int32_t*>(p);
+  p += align256(sizeof(int32_t) * (size_t)(num_seqs + 1));
+  t.cb_start = reinterpret_cast<int32_t*>(p);
+  p += align256(sizeof(int32_t) * (size_t)(num_seqs + 1));
+  t.items = reinterpret_cast<int2*>(p);
+  p += align256(sizeof(int2) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1));
+  t.row_tiles = reinterpret_cast<int64_t*>(p);
+  return t;
+}
+
+// One CTA. Row blocks are ordered by decreasing causal length (I descending), then by sequence,
+// so that the longest rows start first (load balance of the triangular work).
+__global__ void build_tables_kernel(const int32_t* __restrict__ cu, int num_seqs, int B,
+                                    int32_t max_nb, SeqTables t) {
+  if (threadIdx.x == 0) {
+    int32_t rb = 0, cb = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+      int32_t L = cu[s + 1] - cu[s];
+      int32_t nb = (L + B - 1) / B;
+      t.nb[s] = nb;
+      t.rb_start[s] = rb;
+      t.cb_start[s] = cb;
+      rb += nb;
+      cb += nb * (nb + 1) / 2;
+    }
+    t.rb_start[num_seqs] = rb;
+    t.cb_start[num_seqs] = cb;
+  }
+  __syncthreads();
+  for (int I = threadIdx.x; I < max_nb; I += blockDim.x) {
+    int32_t base = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+      int32_t e = t.nb[s] - 1 - I;
+      base += e > 0 ? e : 0;
+    }
+    int32_t c = 0;
+    for (int s = 0; s < num_seqs; ++s)
+      if (t.nb[s] > I) t.items[base + c++] = make_int2(s, I);
+  }
+}
+
+int launch_build_tables(const int32_t* cu_seqlens, int num_seqs, int B, int32_t max_nb,
+                        SeqTables t, cudaStream_t stream) {
+  build_tables_kernel<<<1, 256, 0, stream>>>(cu_seqlens, num_seqs, B, max_nb, t);
+  IAMAP_LAUNCH_CHECK("build_tables_kernel");
+  return IAMAP_OK;
+}
+
+}  // namespace iamap
+
+using namespace iamap;
+
+extern "C" int iamap_version(void) { return (0 << 16) | 1; }
+
+extern "C" const char* iamap_last_error(void) { return g_last_error; }
+
+extern "C" int iamap_device_status(void* stream, int* status) {
+  clear_error();
+  if (!status) return set_error(IAMAP_ERR_INVALID_ARG, "status is null");
+  DeviceContext* c = device_context();
+  if (!c) return IAMAP_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  IAMAP_CUDA_CHECK(cudaStreamSynchronize(st));
+  unsigned int h = 0;
+  IAMAP_CUDA_CHECK(cudaMemcpyAsync(&h, c->status, sizeof(h), cudaMemcpyDeviceToHost, st));
+  IAMAP_CUDA_CHECK(cudaMemsetAsync(c->status, 0, sizeof(unsigned int), st));
+  IAMAP_CUDA_CHECK(cudaStreamSynchronize(st));
+  *status = (int)h;
+  return IAMAP_OK;
+}
+
+extern "C" int iamap_plan(const int32_t* cu_seqlens_host, int num_seqs, int B,
+                          int64_t* num_rowblocks, int64_t* num_causal_blocks,
+                          int32_t* max_blocks_per_seq) {
+  clear_error();
+  Plan p;
+  int rc = make_plan(cu_seqlens_host, num_seqs, B, -1, &p);
+  if (rc) return rc;
+  if (num_rowblocks) *num_rowblocks = p.num_rowblocks;
+  if (num_causal_blocks) *num_causal_blocks = p.num_causal_blocks;
+  if (max_blocks_per_seq) *max_blocks_per_seq = p.max_nb;
+  return IAMAP_OK;
+}
+
+extern "C" size_t iamap_compress_workspace_bytes(int num_seqs, int64_t num_rowblocks) {
+  if (num_seqs < 1 || num_rowblocks < 0) return 0;
+  return seq_tables_bytes(num_seqs, num_rowblocks);
+}

@@ -1,0 +1,227 @@
+"""Python binding of libiamap (ctypes): argument marshalling only.
+
+Every function here has the name and argument order of the C entry point in include/iamap.h.
+Tensors are torch tensors on the current CUDA device (their data pointers are passed); the CUDA
+stream is torch's current stream unless one is given. Nothing is computed in Python: every step
+runs in the library's kernels. If libiamap.so is missing or fails to load, importing this module
+raises ImportError -- there is no fallback.
+
+Small helpers (``alloc_*``) allocate output buffers with torch in the shapes the C ABI documents.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libiamap.so")
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError("libiamap.so not found at %s: build it with "
+                      "`python -m cross_model_attention_map_b200.build`" % _LIB_PATH)
+try:
+    _lib = ctypes.CDLL(_LIB_PATH)
+except OSError as e:  # pragma: no cover - exercised only on broken installs
+    raise ImportError("libiamap.so failed to load: %s" % e) from e
+
+LIB_PATH = _LIB_PATH
+
+IAMAP_OK = 0
+IAMAP_DEV_CAPACITY = 1
+IAMAP_DEV_TIMEOUT = 2
+IAMAP_DEV_BAD_INDEX = 4
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+_SIGS = {
+    "iamap_version": (_I, []),
+    "iamap_last_error": (ctypes.c_char_p, []),
+    "iamap_device_status": (_I, [_P, ctypes.POINTER(_I)]),
+    "iamap_plan": (_I, [_P, _I, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
+                        ctypes.POINTER(ctypes.c_int32)]),
+    "iamap_compress_workspace_bytes": (_SZ, [_I, _I64]),
+    "iamap_compress_stats": (_I, [_P, _P, _P, _P, _I, _I64, _I, _I, _I, _F, _I, _F,
+                                  _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "iamap_compress_extract": (_I, [_P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _F,
+                                    _P, _P, _P, _P, _P, _P, _P, _I64, _P, _SZ, _P]),
+    "iamap_compress": (_I, [_P, _P, _P, _P, _I, _I64, _I, _I, _I, _F, _I, _F,
+                            _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _SZ, _P]),
+    "iamap_mapped_av": (_I, [_P, _P, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _I64, _P, _I, _P,
+                             _I, _P, _P, _SZ, _P]),
+    "iamap_mapped_av_paged_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+    "iamap_mapped_av_paged": (_I, [_P, _I, _P, _P, _I64, _P, _I, _I, _P, _P, _I, _I, _I, _I,
+                                   _P, _P, _SZ, _P]),
+    "iamap_head_match_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+    "iamap_head_match": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ,
+                              _P]),
+}
+
+EXPORTED = tuple(_SIGS)
+
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class IamapError(RuntimeError):
+    def __init__(self, fn, code):
+        msg = _lib.iamap_last_error().decode(errors="replace")
+        super().__init__("%s returned %d: %s" % (fn, code, msg))
+        self.code = code
+
+
+def _check(fn, rc):
+    if rc != IAMAP_OK:
+        raise IamapError(fn, rc)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _host_i32(a):
+    """Host int32 buffer (numpy array, list or CPU tensor) -> (ctypes pointer, keep-alive)."""
+    t = torch.as_tensor(a, dtype=torch.int32).cpu().contiguous()
+    return ctypes.c_void_p(t.data_ptr()), t
+
+
+# ------------------------------------------------------------------------------------------------
+
+def iamap_version() -> int:
+    return _lib.iamap_version()
+
+
+def iamap_last_error() -> str:
+    return _lib.iamap_last_error().decode(errors="replace")
+
+
+def iamap_device_status(stream=None) -> int:
+    st = _I(0)
+    _check("iamap_device_status", _lib.iamap_device_status(_stream(stream), ctypes.byref(st)))
+    return st.value
+
+
+def iamap_plan(cu_seqlens_host, num_seqs, B):
+    p, keep = _host_i32(cu_seqlens_host)
+    nrb, ncb, mx = _I64(0), _I64(0), ctypes.c_int32(0)
+    _check("iamap_plan", _lib.iamap_plan(p, num_seqs, B, ctypes.byref(nrb), ctypes.byref(ncb),
+                                         ctypes.byref(mx)))
+    del keep
+    return nrb.value, ncb.value, mx.value
+
+
+def iamap_compress_workspace_bytes(num_seqs, num_rowblocks) -> int:
+    return _lib.iamap_compress_workspace_bytes(num_seqs, num_rowblocks)
+
+
+def iamap_compress_stats(q, k, cu_seqlens, cu_seqlens_host, num_seqs, n, H_s, d, B, tau,
+                         bias_window, bias_value, lse, mass, headmask_dense, row_ptr, col_idx,
+                         headmask, val_off, counts, ws, stream=None):
+    cp, keep = _host_i32(cu_seqlens_host)
+    _check("iamap_compress_stats", _lib.iamap_compress_stats(
+        _ptr(q), _ptr(k), _ptr(cu_seqlens), cp, num_seqs, n, H_s, d, B, tau, bias_window,
+        bias_value, _ptr(lse), _ptr(mass), _ptr(headmask_dense), _ptr(row_ptr), _ptr(col_idx),
+        _ptr(headmask), _ptr(val_off), _ptr(counts), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+    del keep
+
+
+def iamap_compress_extract(q, k, cu_seqlens, cu_seqlens_host, num_seqs, n, H_s, d, B,
+                           bias_window, bias_value, lse, row_ptr, col_idx, headmask, val_off,
+                           counts, vals, vals_capacity_tiles, ws, stream=None):
+    cp, keep = _host_i32(cu_seqlens_host)
+    _check("iamap_compress_extract", _lib.iamap_compress_extract(
+        _ptr(q), _ptr(k), _ptr(cu_seqlens), cp, num_seqs, n, H_s, d, B, bias_window, bias_value,
+        _ptr(lse), _ptr(row_ptr), _ptr(col_idx), _ptr(headmask), _ptr(val_off), _ptr(counts),
+        _ptr(vals), vals_capacity_tiles, _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+    del keep
+
+
+def iamap_compress(q, k, cu_seqlens, cu_seqlens_host, num_seqs, n, H_s, d, B, tau, bias_window,
+                   bias_value, lse, mass, headmask_dense, row_ptr, col_idx, headmask, val_off,
+                   counts, vals, vals_capacity_tiles, ws, stream=None):
+    cp, keep = _host_i32(cu_seqlens_host)
+    _check("iamap_compress", _lib.iamap_compress(
+        _ptr(q), _ptr(k), _ptr(cu_seqlens), cp, num_seqs, n, H_s, d, B, tau, bias_window,
+        bias_value, _ptr(lse), _ptr(mass), _ptr(headmask_dense), _ptr(row_ptr), _ptr(col_idx),
+        _ptr(headmask), _ptr(val_off), _ptr(counts), _ptr(vals), vals_capacity_tiles, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def iamap_mapped_av(cu_seqlens, cu_seqlens_host, num_seqs, n, B, H_s, row_ptr, col_idx, headmask,
+                    val_off, vals, vals_capacity_tiles, W, H_r, v, d_v, out, ws, stream=None):
+    cp, keep = _host_i32(cu_seqlens_host)
+    _check("iamap_mapped_av", _lib.iamap_mapped_av(
+        _ptr(cu_seqlens), cp, num_seqs, n, B, H_s, _ptr(row_ptr), _ptr(col_idx), _ptr(headmask),
+        _ptr(val_off), _ptr(vals), vals_capacity_tiles, _ptr(W), H_r, _ptr(v), d_v, _ptr(out),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def iamap_mapped_av_paged_workspace_bytes(batch, H_r, d_v, max_ctx, page_size) -> int:
+    return _lib.iamap_mapped_av_paged_workspace_bytes(batch, H_r, d_v, max_ctx, page_size)
+
+
+def iamap_mapped_av_paged(p_rows, ctx_stride, W, v_pages, num_pages, page_table, max_pages,
+                          page_size, ctx_lens, ctx_lens_host, batch, H_s, H_r, d_v, out, ws,
+                          stream=None):
+    cp, keep = _host_i32(ctx_lens_host)
+    _check("iamap_mapped_av_paged", _lib.iamap_mapped_av_paged(
+        _ptr(p_rows), ctx_stride, _ptr(W), _ptr(v_pages), num_pages, _ptr(page_table), max_pages,
+        page_size, _ptr(ctx_lens), cp, batch, H_s, H_r, d_v, _ptr(out), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def iamap_head_match_workspace_bytes(L_s, H_small, L_l, H_large, n_used) -> int:
+    return _lib.iamap_head_match_workspace_bytes(L_s, H_small, L_l, H_large, n_used)
+
+
+def iamap_head_match(q_small, k_small, L_s, H_small, d_small, q_large, k_large, L_l, H_large,
+                     d_large, n, n_used, argmax, sim, ws, stream=None):
+    _check("iamap_head_match", _lib.iamap_head_match(
+        _ptr(q_small), _ptr(k_small), L_s, H_small, d_small, _ptr(q_large), _ptr(k_large), L_l,
+        H_large, d_large, n, n_used, _ptr(argmax), _ptr(sim), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+# ------------------------------------------------------------------------------------------------
+# Buffer helpers (torch allocations in the documented shapes)
+# ------------------------------------------------------------------------------------------------
+
+def alloc_compress_outputs(n, H_s, num_rowblocks, num_causal_blocks, device="cuda"):
+    """lse, mass, headmask_dense, row_ptr, col_idx, headmask, val_off, counts."""
+    i64 = torch.int64
+    return dict(
+        lse=torch.empty(H_s, n, dtype=torch.float32, device=device),
+        mass=torch.empty(H_s, num_causal_blocks, dtype=torch.float32, device=device),
+        headmask_dense=torch.empty(num_causal_blocks, dtype=i64, device=device),
+        row_ptr=torch.empty(num_rowblocks + 1, dtype=torch.int32, device=device),
+        col_idx=torch.empty(max(num_causal_blocks, 1), dtype=torch.int32, device=device),
+        headmask=torch.empty(max(num_causal_blocks, 1), dtype=i64, device=device),
+        val_off=torch.empty(max(num_causal_blocks, 1), dtype=i64, device=device),
+        counts=torch.zeros(2, dtype=i64, device=device),
+    )
+
+
+def alloc_workspace(nbytes, device="cuda"):
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)

@@ -1,0 +1,109 @@
+"""Buffer management around the C ABI for one mapped prefill layer (allocation and calls only).
+
+``PrefillLayer`` owns the device buffers of one (sender layer, receiver layer) pair with fixed
+packed sequence lengths and runs the hot path through libiamap:
+
+    compress(q, k)          -> lse, block masses, BSR index and bf16 tiles (no host sync)
+    mapped_av(W, v)         -> out [n, H_r, d_v]
+    step(q, k, W, v)        -> both
+
+The value buffer is sized for the worst case (every head keeps every causal block) unless a
+capacity is given, so the step needs no host synchronisation.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import iamap as C
+
+
+class PrefillLayer:
+    def __init__(self, seqlens, H_s, d, H_r, d_v, tau, bias_window=0, bias_value=0.0, B=64,
+                 capacity_tiles=None, device="cuda"):
+        self.seqlens = [int(x) for x in seqlens]
+        self.num_seqs = len(self.seqlens)
+        cu = [0]
+        for L in self.seqlens:
+            cu.append(cu[-1] + L)
+        self.cu_host = torch.tensor(cu, dtype=torch.int32)
+        self.cu = self.cu_host.to(device)
+        self.n = cu[-1]
+        self.H_s, self.d, self.H_r, self.d_v, self.B = H_s, d, H_r, d_v, B
+        self.tau, self.bias_window, self.bias_value = float(tau), int(bias_window), float(bias_value)
+        self.nrb, self.ncb, self.max_nb = C.iamap_plan(self.cu_host, self.num_seqs, B)
+        self.bufs = C.alloc_compress_outputs(self.n, H_s, self.nrb, self.ncb, device)
+        cap = H_s * self.ncb if capacity_tiles is None else int(capacity_tiles)
+        self.capacity = cap
+        self.vals = torch.empty(max(cap, 1), B, B, dtype=torch.bfloat16, device=device)
+        self.ws = C.alloc_workspace(C.iamap_compress_workspace_bytes(self.num_seqs, self.nrb),
+                                    device)
+        self.out = torch.empty(self.n, H_r, d_v, dtype=torch.float32, device=device)
+
+    def compress(self, q, k, stream=None):
+        b = self.bufs
+        C.iamap_compress(q, k, self.cu, self.cu_host, self.num_seqs, self.n, self.H_s, self.d,
+                         self.B, self.tau, self.bias_window, self.bias_value, b["lse"], b["mass"],
+                         b["headmask_dense"], b["row_ptr"], b["col_idx"], b["headmask"],
+                         b["val_off"], b["counts"], self.vals, self.capacity, self.ws, stream)
+
+    def mapped_av(self, W, v, stream=None):
+        b = self.bufs
+        C.iamap_mapped_av(self.cu, self.cu_host, self.num_seqs, self.n, self.B, self.H_s,
+                          b["row_ptr"], b["col_idx"], b["headmask"], b["val_off"], self.vals,
+                          self.capacity, W, self.H_r, v, self.d_v, self.out, self.ws, stream)
+
+    def step(self, q, k, W, v, stream=None):
+        self.compress(q, k, stream)
+        self.mapped_av(W, v, stream)
+        return self.out
+
+    def counts(self):
+        """(nnz_blocks, nnz_tiles) -- synchronises."""
+        c = self.bufs["counts"].cpu()
+        return int(c[0]), int(c[1])
+
+
+class DecodeStep:
+    """Buffers of one paged decode step on a mapped layer."""
+
+    def __init__(self, batch, H_s, H_r, d_v, ctx_lens_host, ctx_stride, max_pages, page_size,
+                 num_pages, device="cuda"):
+        self.batch, self.H_s, self.H_r, self.d_v = batch, H_s, H_r, d_v
+        self.ctx_lens_host = torch.as_tensor(ctx_lens_host, dtype=torch.int32).cpu()
+        self.ctx_lens = self.ctx_lens_host.to(device)
+        self.ctx_stride, self.max_pages, self.page_size = ctx_stride, max_pages, page_size
+        self.num_pages = num_pages
+        max_ctx = int(self.ctx_lens_host.max())
+        self.ws = C.alloc_workspace(
+            C.iamap_mapped_av_paged_workspace_bytes(batch, H_r, d_v, max_ctx, page_size), device)
+        self.out = torch.empty(batch, H_r, d_v, dtype=torch.float32, device=device)
+
+    def run(self, p_rows, W, v_pages, page_table, stream=None):
+        C.iamap_mapped_av_paged(p_rows, self.ctx_stride, W, v_pages, self.num_pages, page_table,
+                                self.max_pages, self.page_size, self.ctx_lens, self.ctx_lens_host,
+                                self.batch, self.H_s, self.H_r, self.d_v, self.out, self.ws,
+                                stream)
+        return self.out
+
+
+class HeadMatch:
+    """Buffers of one head-matching calibration."""
+
+    def __init__(self, L_s, H_small, d_small, L_l, H_large, d_large, n, n_used=None,
+                 want_sim=True, device="cuda"):
+        self.dims = (L_s, H_small, d_small, L_l, H_large, d_large)
+        self.n = n
+        self.n_used = n if n_used is None else int(n_used)
+        self.ws = C.alloc_workspace(
+            C.iamap_head_match_workspace_bytes(L_s, H_small, L_l, H_large, self.n_used), device)
+        self.argmax = torch.empty(L_l * H_large, dtype=torch.int32, device=device)
+        self.sim = (torch.empty(L_l * H_large, L_s * H_small, dtype=torch.float32, device=device)
+                    if want_sim else None)
+
+    def run(self, q_small, k_small, q_large, k_large, stream=None):
+        L_s, H_small, d_small, L_l, H_large, d_large = self.dims
+        C.iamap_head_match(q_small, k_small, L_s, H_small, d_small, q_large, k_large, L_l,
+                           H_large, d_large, self.n, self.n_used, self.argmax, self.sim, self.ws,
+                           stream)
+        return self.argmax, self.sim

@@ -1,0 +1,198 @@
+/*
+ * iamap.h -- C ABI of the cross-model attention-map reuse library (libiamap.so, sm_100a).
+ *
+ * The library computes, on one NVIDIA B200, the hot path of reusing one model's attention map in
+ * another model's attention output:
+ *
+ *   compress     a sender model's causal softmax attention, per head, turned into a block-sparse
+ *                (BSR) map: first block-level probability mass, then the extraction of the blocks
+ *                kept by cumulative mass, with no dense n x n matrix ever formed.
+ *                ("PKU MapFlow: cross-model attention map reuse" news page, storage-and-execution
+ *                part, first component.)
+ *   mapped_av    for every kept block, mix the sender heads by an H_r x H_s matrix W on chip,
+ *                multiply by the receiver's V and accumulate the output, with no dense receiver
+ *                map. (Same page, third component; the head mapping as a learned linear
+ *                combination of sender heads is in its layer/head-mapping paragraph.)
+ *   mapped_av_paged  the decode form: one query row per sequence, sender rows given, V in a paged
+ *                cache. ("IAM: Efficient Inference through Attention Mapping between
+ *                Different-scale LLMs" notes, Method section 4, decode bullet.)
+ *   head_match   IAM's calibration: cosine similarity of flattened causal attention maps of every
+ *                large-model head with every small-model head, then the most similar small head
+ *                per large head. (IAM notes, Method sections 1 and 4.)
+ *
+ * Conventions (all entry points):
+ *   - Return 0 (IAMAP_OK) or a negative IAMAP_ERR_* code; iamap_last_error() gives a
+ *     thread-local message for the last failure. No C++ exception crosses this boundary.
+ *   - Tensor pointers are DEVICE pointers owned by the caller unless the name ends in _host.
+ *     The library never frees or keeps them. bf16 tensors are passed as void* (IEEE bfloat16).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Work is enqueued
+ *     asynchronously on it; no entry point synchronises the stream except iamap_device_status.
+ *   - The library keeps one lazily created context per device: a device status word that kernels
+ *     set on a detected error (capacity exceeded, bounded wait expired, malformed index). Read and
+ *     clear it with iamap_device_status.
+ *   - Only block size B = 64 is implemented (IAMAP_ERR_UNSUPPORTED otherwise). Head dims d, d_v
+ *     must be 64 or 128. Sender heads H_s <= 64 (one bit per head in the head masks).
+ *
+ * Layouts:
+ *   q, k      bf16 [n, H_s, d]     token-major, packed sequences (cu_seqlens, int32 [S+1])
+ *   v         bf16 [n, H_r, d_v]
+ *   W         fp32 [H_r, H_s]      row r mixes the sender heads for receiver head r
+ *   lse       fp32 [H_s, n]        natural-log row log-sum-exp of the sender's scaled logits
+ *   Causal blocks: sequence s has nb_s = ceil(L_s / B) row blocks; row block I has column blocks
+ *   J = 0..I. Global row-block index rb = rb_start[s] + I; causal-block index
+ *   cb = cb_start[s] + I*(I+1)/2 + J (both enumerations sequence-major, as iamap_plan reports).
+ *   mass      fp32 [H_s, num_causal_blocks]  summed probability of each (head, causal block)
+ *   headmask_dense u64 [num_causal_blocks]   bit h set = sender head h keeps that block
+ *   BSR (union over heads, per row block, column blocks ascending):
+ *     row_ptr  int32 [num_rowblocks + 1]
+ *     col_idx  int32 [nnz_blocks]   column-block index J (local to the sequence)
+ *     headmask u64   [nnz_blocks]   present sender heads
+ *     val_off  int64 [nnz_blocks]   tile index of the first present head; the tiles of the
+ *                                   present heads follow in increasing head order
+ *     vals     bf16  [tiles, B, B]  row-major probability tiles; causally masked entries and rows
+ *                                   past the sequence end are 0
+ *   out       fp32 [n, H_r, d_v]
+ */
+#ifndef IAMAP_H
+#define IAMAP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define IAMAP_OK                0
+#define IAMAP_ERR_INVALID_ARG  (-1)   /* null pointer, bad size or shape */
+#define IAMAP_ERR_UNSUPPORTED  (-2)   /* valid but not implemented (B != 64, d not 64/128, ...) */
+#define IAMAP_ERR_CAPACITY     (-3)   /* an output buffer is too small for the data */
+#define IAMAP_ERR_CUDA         (-4)   /* a CUDA runtime call or launch failed */
+#define IAMAP_ERR_TIMEOUT      (-5)   /* a bounded device-side wait expired */
+#define IAMAP_ERR_WORKSPACE    (-6)   /* workspace pointer null or smaller than required */
+
+/* Device status bits (iamap_device_status). */
+#define IAMAP_DEV_CAPACITY   1
+#define IAMAP_DEV_TIMEOUT    2
+#define IAMAP_DEV_BAD_INDEX  4
+
+/* Library version, (major << 16) | minor. */
+int iamap_version(void);
+
+/* Thread-local message of the last failed call on this thread ("" if none). */
+const char* iamap_last_error(void);
+
+/*
+ * Synchronise `stream`, then read and clear the device status word of the current device.
+ * *status receives a bitwise OR of IAMAP_DEV_* (0 = no device-side error since the last read).
+ * Returns IAMAP_ERR_CUDA if the synchronisation itself reports an error.
+ */
+int iamap_device_status(void* stream, int* status);
+
+/*
+ * Planning (host only, no device work). From the host copy of cu_seqlens, report the number of
+ * row blocks, of causal blocks, and the largest row-block count of any sequence.
+ * Errors: IAMAP_ERR_INVALID_ARG if cu_seqlens_host is null, num_seqs < 1, B < 1, or the offsets
+ * decrease.
+ */
+int iamap_plan(const int32_t* cu_seqlens_host, int num_seqs, int B, int64_t* num_rowblocks,
+               int64_t* num_causal_blocks, int32_t* max_blocks_per_seq);
+
+/* Workspace bytes needed by iamap_compress_stats / _extract / iamap_compress / iamap_mapped_av
+ * (scheduling tables). */
+size_t iamap_compress_workspace_bytes(int num_seqs, int64_t num_rowblocks);
+
+/*
+ * Compress, stage 1 (block-level statistics and the kept sets).
+ * For every sender head h and row block: the row-wise log-sum-exp of the scaled causal logits
+ * s_ij = q_i.k_j / sqrt(d) (+ bias_value when 0 <= i - j < bias_window; window 0 = no bias),
+ * the probability mass of every causal column block, and the kept set: the shortest prefix of
+ * the column blocks sorted by decreasing mass (ties: lower J) whose cumulative mass reaches
+ * tau * (valid rows of the block); tau >= 1 keeps every causal block. Then the union BSR index
+ * (row_ptr, col_idx, headmask, val_off) and counts[0] = nnz_blocks, counts[1] = nnz_tiles.
+ * col_idx / headmask / val_off must hold num_causal_blocks entries (the nnz is data-dependent).
+ * Outputs lse, mass, headmask_dense, row_ptr, col_idx, headmask, val_off, counts are written in
+ * full. The only input read on the host is cu_seqlens_host (the same values as cu_seqlens).
+ */
+int iamap_compress_stats(const void* q, const void* k, const int32_t* cu_seqlens,
+                         const int32_t* cu_seqlens_host, int num_seqs, int64_t n, int H_s, int d,
+                         int B, float tau, int bias_window, float bias_value,
+                         float* lse, float* mass, uint64_t* headmask_dense, int32_t* row_ptr,
+                         int32_t* col_idx, uint64_t* headmask, int64_t* val_off, int64_t* counts,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Compress, stage 2 (extraction of the kept blocks). Recomputes each kept (head, row block,
+ * column block) tile of probabilities exp(s_ij - lse_i) from q, k and stage 1's lse, and writes
+ * it as a bf16 B x B tile at its BSR position. A tile whose index is >= vals_capacity_tiles is not
+ * written and sets IAMAP_DEV_CAPACITY in the device status. After the last tile the call also
+ * zero-fills up to 64 further tiles that fit in the capacity (mapped_av may read that far).
+ */
+int iamap_compress_extract(const void* q, const void* k, const int32_t* cu_seqlens,
+                           const int32_t* cu_seqlens_host, int num_seqs, int64_t n, int H_s, int d,
+                           int B, int bias_window, float bias_value, const float* lse,
+                           const int32_t* row_ptr, const int32_t* col_idx, const uint64_t* headmask,
+                           const int64_t* val_off, const int64_t* counts, void* vals,
+                           int64_t vals_capacity_tiles, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Compress, both stages back to back on `stream`, with no host synchronisation (the tile count
+ * stays on the device; a shortfall of vals_capacity_tiles is reported through the device status).
+ */
+int iamap_compress(const void* q, const void* k, const int32_t* cu_seqlens,
+                   const int32_t* cu_seqlens_host, int num_seqs, int64_t n, int H_s, int d, int B,
+                   float tau, int bias_window, float bias_value, float* lse, float* mass,
+                   uint64_t* headmask_dense, int32_t* row_ptr, int32_t* col_idx, uint64_t* headmask,
+                   int64_t* val_off, int64_t* counts, void* vals, int64_t vals_capacity_tiles,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Mapped attention output: for each row block and each stored column block J,
+ *   P_r = sum_s W[r, s] * Pt_s   (absent heads contribute 0; no renormalisation),
+ *   out_r[rows of the block] += P_r . V_r[rows of J],
+ * for all receiver heads r < H_r; `out` is overwritten. vals_capacity_tiles bounds every tile
+ * read (indices beyond it set IAMAP_DEV_BAD_INDEX).
+ */
+int iamap_mapped_av(const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int num_seqs,
+                    int64_t n, int B, int H_s, const int32_t* row_ptr, const int32_t* col_idx,
+                    const uint64_t* headmask, const int64_t* val_off, const void* vals,
+                    int64_t vals_capacity_tiles, const float* W, int H_r, const void* v, int d_v,
+                    float* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Decode step on a mapped layer: one query row per sequence b.
+ *   out[b, r, :] = sum_{j < ctx_lens[b]} (sum_s W[r, s] * p_rows[b, s, j]) * V[b, j, r, :]
+ * p_rows  fp32 [batch, H_s, ctx_stride]  the sender's attention rows
+ * v_pages bf16 [num_pages, page_size, H_r, d_v]; token j of sequence b lives in page
+ *         page_table[b * max_pages + j / page_size], slot j % page_size.
+ * out     fp32 [batch, H_r, d_v]. ws: iamap_mapped_av_paged_workspace_bytes bytes (split partial
+ * sums). Page indices outside [0, num_pages) set IAMAP_DEV_BAD_INDEX and are skipped.
+ */
+size_t iamap_mapped_av_paged_workspace_bytes(int batch, int H_r, int d_v, int max_ctx,
+                                             int page_size);
+int iamap_mapped_av_paged(const float* p_rows, int ctx_stride, const float* W,
+                          const void* v_pages, int64_t num_pages, const int32_t* page_table,
+                          int max_pages, int page_size, const int32_t* ctx_lens,
+                          const int32_t* ctx_lens_host, int batch, int H_s, int H_r, int d_v,
+                          float* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Head matching (calibration). q_small / k_small bf16 [L_s, n, H_small, d_small];
+ * q_large / k_large bf16 [L_l, n, H_large, d_large]. Each head's map is the causal softmax of
+ * q k^T / sqrt(d) over the first n_used tokens (n_used <= n; the prompt truncation tau_t).
+ * sim (optional, may be NULL) fp32 [L_l * H_large, L_s * H_small]: cosine of the flattened maps.
+ * argmax int32 [L_l * H_large]: the small head (layer * H_small + head) of highest cosine,
+ * lowest index on ties. ws: iamap_head_match_workspace_bytes bytes (the bf16 maps, norms and
+ * the similarity accumulator).
+ */
+size_t iamap_head_match_workspace_bytes(int L_s, int H_small, int L_l, int H_large, int n_used);
+int iamap_head_match(const void* q_small, const void* k_small, int L_s, int H_small, int d_small,
+                     const void* q_large, const void* k_large, int L_l, int H_large, int d_large,
+                     int n, int n_used, int32_t* argmax, float* sim, void* ws, size_t ws_bytes,
+                     void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IAMAP_H */

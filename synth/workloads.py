@@ -224,7 +224,9 @@ def make_decode(batch=4, ctx=8704, H_s=14, H_r=64, d_v=128, page_size=16, sink_w
     g[:, :, 0] *= sink_weight
     for b in range(batch):
         g[b, :, ctx_lens[b]:] = 0.0
-    p_rows = (g / g.sum(axis=2, keepdims=True)).astype(np.float32)
+    den = g.sum(axis=2, keepdims=True)
+    den[den == 0] = 1.0
+    p_rows = (g / den).astype(np.float32)
     assign = rng.integers(0, H_s, size=H_r).astype(np.int32)
     W = np.zeros((H_r, H_s), dtype=np.float32)
     W[np.arange(H_r), assign] = 1.0

@@ -1,0 +1,87 @@
+"""CPU checks of the C-ABI library: it loads, exports every entry point declared in
+include/iamap.h, and rejects bad arguments on the host (no GPU needed, no compute call)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "iamap.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from cross_model_attention_map_b200 import build
+    build.build()
+    from cross_model_attention_map_b200 import iamap
+    return iamap
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(iamap_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("iamap_compress", "iamap_compress_stats", "iamap_compress_extract",
+              "iamap_mapped_av", "iamap_mapped_av_paged", "iamap_head_match"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (iamap_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(raw, n)
+    # the binding wraps every declared function under the same name
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_plan_counts(lib):
+    nrb, ncb, mx = lib.iamap_plan([0, 4096, 12288, 24576, 40960], 4, 64)
+    assert (nrb, ncb, mx) == (640, 2080 + 8256 + 18528 + 32896, 256)
+    nrb, ncb, mx = lib.iamap_plan([0, 1, 65, 130], 3, 64)
+    assert (nrb, ncb, mx) == (1 + 1 + 2, 1 + 1 + 3, 2)
+
+
+def test_plan_rejects_bad_offsets(lib):
+    with pytest.raises(lib.IamapError) as e:
+        lib.iamap_plan([0, 10, 5], 2, 64)
+    assert e.value.code == -1
+    with pytest.raises(lib.IamapError):
+        lib.iamap_plan([3, 10], 1, 64)
+
+
+def test_host_validation_without_gpu(lib):
+    """Unsupported block size and null pointers are refused before any device work."""
+    raw = lib._lib
+    rc = raw.iamap_compress_stats(None, None, None, None, 1, 64, 8, 64, 32, 0.9, 0, 0.0, None,
+                                  None, None, None, None, None, None, None, None, 0, None)
+    assert rc == -2 and "B = 64" in lib.iamap_last_error()
+    rc = raw.iamap_compress_stats(None, None, None, None, 1, 64, 8, 64, 64, 0.9, 0, 0.0, None,
+                                  None, None, None, None, None, None, None, None, 0, None)
+    assert rc == -1
+    rc = raw.iamap_mapped_av_paged(None, 0, None, None, 0, None, 0, 16, None, None, 1, 1, 1, 8,
+                                   None, None, 0, None)
+    assert rc == -1
+    rc = raw.iamap_head_match(None, None, 1, 1, 64, None, None, 1, 1, 128, 8, 8, None, None, None,
+                              0, None)
+    assert rc == -1
+    st = ctypes.c_int(0)
+    assert raw.iamap_device_status(None, None) == -1
+
+
+def test_workspace_queries(lib):
+    assert lib.iamap_compress_workspace_bytes(4, 640) > 640 * 8
+    assert lib.iamap_head_match_workspace_bytes(24, 14, 8, 64, 1024) > 848 * 136 * 8192
+    assert lib.iamap_mapped_av_paged_workspace_bytes(4, 64, 128, 8704, 16) > 0
