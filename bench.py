@@ -1,0 +1,553 @@
+"""Benchmark of cross-model attention-map reuse on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+A step is one pass of the hot path over one synthetic batch: map_compress (block statistics +
+selection + union index, then extraction of the kept tiles) followed by mapped_av, on the
+packed-prefill workload (default ``varlen40k``: 4 causal sequences of 4096/8192/12288/16384
+tokens = 40960 tokens, sender 40 heads d=128, receiver 32 heads d_v=128, B=64, tau=0.9). Inputs
+are resident in HBM when the timed region starts; Q+K (840 MB) and the block-sparse values
+(~17 GB) exceed the 126 MB L2, so no flush is needed between steps.
+
+Other configs (for measurement of the other kernels): ``tiny``, ``prefill8k``, ``headmatch``
+(head_match, n=1024, 24x14 small / 8x64 large heads), ``decode`` (paged decode, batch 4,
+context 8704).
+
+Multi-GPU (torchrun): every rank runs its own full batch (independent problems, no data-path
+collective, weak scaling); rank 0 prints value = tokens of all ranks / max time over ranks.
+
+``--impl reference`` times the float64 CPU oracle (rank 0 only) on a bounded sample of the same
+workload, in the same metric.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mapped-attention tokens/s at n=32k (1 B200); achieved % HBM / tensor roofline"
+PROFILES = os.path.join(ROOT, "profiles")
+
+CONFIG_TEXT = {
+    "varlen40k": ("varlen40k: 4 packed causal sequences 4096/8192/12288/16384 (40960 tokens), "
+                  "sender H_s=40 d=128, receiver H_r=32 d_v=128, B=64, tau=0.9, sink; "
+                  "compress + mapped_av"),
+    "prefill8k": ("prefill8k: 1 causal sequence n=8192, H_s=32 d=128, H_r=24 d_v=128, B=64, "
+                  "tau=0.95, sink, local bias +2.0 on |i-j|<128; compress + mapped_av"),
+    "tiny": "tiny: n=512, H_s=8 d=64, H_r=4 d_v=64, B=64, tau=0.95, sink; compress + mapped_av",
+    "headmatch": ("headmatch: n=1024, small 24 layers x 14 heads d=64, large 8 layers x 64 heads "
+                  "d=128, planted noisy copies; head_match"),
+    "decode": ("decode: batch 4, q_len 1, context 8704, sender 14 heads, receiver 64 heads "
+               "d_v=128, one-hot W, 16-token pages; mapped_av_paged"),
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                source="fallback")
+
+
+def src_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "cross_model_attention_map_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel, files):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current source."""
+    p = os.path.join(PROFILES, "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d or d.get("source_sha") != src_sha(files):
+        return None
+    return d.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ------------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 5.0 and self.proc.poll() is None:
+                time.sleep(0.02)
+            self.lines.clear()   # samples from before the timed region
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# Distributed plumbing
+# ------------------------------------------------------------------------------------------------
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample
+# ------------------------------------------------------------------------------------------------
+
+def oracle_sample_prefill(wl, budget_s=20.0, seed=0):
+    """Oracle compress + mapped_av on random row blocks (all sender and receiver heads) until the
+    budget is used. Returns (tokens/s, rows, seconds, sample text)."""
+    import oracle as O
+    lay = O.causal_layout(wl.seqlens, wl.B)
+    rng = np.random.default_rng(seed)
+    blocks = [(s, I) for s in range(len(wl.seqlens)) for I in range(lay.nb[s])]
+    order = rng.permutation(len(blocks))
+    rows = 0
+    t0 = time.perf_counter()
+    done = 0
+    for idx in order:
+        s, I = blocks[idx]
+        st = {h: O.rowblock_stats(wl.q, wl.k, wl.cu_seqlens, s, h, I, wl.B, wl.tau,
+                                  wl.bias_window, wl.bias_value) for h in range(wl.H_s)}
+        O.mapped_av_rows(wl, s, I, lambda h: st[h].kept, lambda h: st[h])
+        rows += st[0].R
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    text = ("%d uniformly drawn row blocks of %d (%d query rows, all %d sender and %d receiver "
+            "heads): float64 compress + mapped_av" % (done, len(blocks), rows, wl.H_s, wl.H_r))
+    return rows / dt, rows, dt, text
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arms
+# ------------------------------------------------------------------------------------------------
+
+def bf16_dev(bits, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def bench_prefill(args, world, rank, local, peaks):
+    import torch
+    from synth import prefill_config
+    from cross_model_attention_map_b200 import iamap as C
+    from cross_model_attention_map_b200.runner import PrefillLayer
+
+    dev = torch.device("cuda", local)
+    wl = prefill_config(args.config, seed=rank)
+    q, k, v = bf16_dev(wl.q, dev), bf16_dev(wl.k, dev), bf16_dev(wl.v, dev)
+    W = torch.from_numpy(wl.W).to(dev)
+    layer = PrefillLayer(wl.seqlens, wl.H_s, wl.d, wl.H_r, wl.d_v, wl.tau, wl.bias_window,
+                         wl.bias_value, device=dev)
+    stream = torch.cuda.current_stream()
+    b = layer.bufs
+
+    def stats():
+        C.iamap_compress_stats(q, k, layer.cu, layer.cu_host, layer.num_seqs, layer.n, wl.H_s,
+                               wl.d, wl.B, wl.tau, wl.bias_window, wl.bias_value, b["lse"],
+                               b["mass"], b["headmask_dense"], b["row_ptr"], b["col_idx"],
+                               b["headmask"], b["val_off"], b["counts"], layer.ws, stream)
+
+    def extract():
+        C.iamap_compress_extract(q, k, layer.cu, layer.cu_host, layer.num_seqs, layer.n, wl.H_s,
+                                 wl.d, wl.B, wl.bias_window, wl.bias_value, b["lse"],
+                                 b["row_ptr"], b["col_idx"], b["headmask"], b["val_off"],
+                                 b["counts"], layer.vals, layer.capacity, layer.ws, stream)
+
+    def mapped():
+        layer.mapped_av(W, v, stream)
+
+    # launches of our kernels per step: stats call 5 (tables, stats, row count/scan/fill),
+    # extract call 3 (tables, extract, zero tail), mapped_av call 2 (tables, mapped_av)
+    launches_per_step = 10
+    for _ in range(args.warmup):
+        stats(); extract(); mapped()
+    torch.cuda.synchronize()
+    assert C.iamap_device_status(stream) == 0
+    nnz_blocks, nnz_tiles = layer.counts()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream); stats()
+        ev[i][1].record(stream); extract()
+        ev[i][2].record(stream); mapped()
+        ev[i][3].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    barrier(world)
+    ms_local = t_start.elapsed_time(t_end) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    t_stats = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    t_extract = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    t_av = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
+    assert C.iamap_device_status(stream) == 0
+
+    n = layer.n
+    tokens_total = n * world
+    value = tokens_total / (ms * 1e-3)
+
+    # algorithmic work per launch
+    causal_pairs = sum(L * (L + 1) // 2 for L in wl.seqlens)
+    qk_flops = 2.0 * wl.d * causal_pairs * wl.H_s                     # one causal QK^T
+    exps = float(causal_pairs) * wl.H_s
+    av_bytes = (8192.0 * nnz_tiles + 20.0 * nnz_blocks + 4.0 * (layer.nrb + 1)
+                + 2.0 * n * wl.H_r * wl.d_v + 4.0 * n * wl.H_r * wl.d_v + 4.0 * wl.H_r * wl.H_s)
+    extract_bytes = 8192.0 * nnz_tiles + 2.0 * 2 * n * wl.H_s * wl.d + 4.0 * n * wl.H_s
+    kernels = {
+        "compress_stats": {"ms": t_stats, "bound": "tensor", "flops": qk_flops,
+                           "tflops": qk_flops / (t_stats * 1e-3) / 1e12, "exps": exps},
+        "compress_extract": {"ms": t_extract, "bound": "hbm", "bytes": extract_bytes,
+                             "gbs": extract_bytes / (t_extract * 1e-3) / 1e9,
+                             "tflops_qk_recompute": qk_flops * nnz_tiles / (wl.H_s * layer.ncb)
+                             / (t_extract * 1e-3) / 1e12},
+        "mapped_av": {"ms": t_av, "bound": "hbm", "bytes": av_bytes,
+                      "gbs": av_bytes / (t_av * 1e-3) / 1e9},
+    }
+    dom = max(kernels, key=lambda kname: kernels[kname]["ms"])
+    kd = kernels[dom]
+    if kd["bound"] == "hbm":
+        achieved = kd["gbs"]
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    else:
+        achieved = kd["tflops"]
+        peak = peaks["bf16_tflops_sustained"]
+        unit = "TFLOP/s"
+    files = {"mapped_av": ["mapped_av.cu"], "compress_stats": ["compress.cu", "qk_tile.cuh"],
+             "compress_extract": ["compress.cu", "qk_tile.cuh"]}[dom]
+    roofline = {"kernel": dom, "bound": kd["bound"], "achieved": round(achieved, 2),
+                "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
+                "traffic": load_traffic(dom, files),
+                "peak_source": peaks["source"] + (" sustained bf16" if unit == "TFLOP/s" else " HBM copy")}
+
+    # end to end through the public API with host buffers (pinned), per step: H2D of q, k, v, W,
+    # cu_seqlens; the step; D2H of the output.
+    hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True); hq.copy_(q)
+    hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True); hk.copy_(k)
+    hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True); hv.copy_(v)
+    hW = torch.empty(W.shape, dtype=W.dtype, pin_memory=True); hW.copy_(W)
+    hcu = torch.empty(layer.cu.shape, dtype=torch.int32, pin_memory=True); hcu.copy_(layer.cu)
+    hout = torch.empty(layer.out.shape, dtype=torch.float32, pin_memory=True)
+    e2e_steps = max(2, min(args.steps, 5))
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True); W.copy_(hW, non_blocking=True)
+        layer.cu.copy_(hcu, non_blocking=True)
+        layer.step(q, k, W, v, stream)
+        hout.copy_(layer.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hW, hcu))
+    d2h = hout.numel() * hout.element_size()
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; the configuration's shapes and distributions)",
+        "config": {"workload": CONFIG_TEXT[args.config], "tokens_per_gpu": n,
+                   "nnz_blocks": nnz_blocks, "nnz_tiles": nnz_tiles,
+                   "kept_tile_density": round(nnz_tiles / (wl.H_s * layer.ncb), 4),
+                   "l2": "inputs larger than L2 (Q+K %.0f MB, BSR values %.1f GB); no flush"
+                         % (4.0 * n * wl.H_s * wl.d / 1e6, 8192.0 * nnz_tiles / 1e9),
+                   "parallelism": "dp%d (independent batches per GPU, no collective)" % world},
+        "kernels": {kk: {x: (round(y, 4) if isinstance(y, float) else y) for x, y in kv.items()}
+                    for kk, kv in kernels.items()},
+        "roofline": roofline,
+        "clocks": clocks,
+        "e2e": {"value": round(tokens_total / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    return line, wl
+
+
+def bench_decode(args, world, rank, local, peaks):
+    import torch
+    from synth import decode_config
+    from cross_model_attention_map_b200 import iamap as C
+    from cross_model_attention_map_b200.runner import DecodeStep
+
+    dev = torch.device("cuda", local)
+    dw = decode_config(seed=rank)
+    st = DecodeStep(dw.batch, dw.H_s, dw.H_r, dw.d_v, dw.ctx_lens, dw.p_rows.shape[2],
+                    dw.page_table.shape[1], dw.page_size, dw.v_pages.shape[0], device=dev)
+    p = torch.from_numpy(dw.p_rows).to(dev)
+    W = torch.from_numpy(dw.W).to(dev)
+    vp = bf16_dev(dw.v_pages, dev)
+    pt = torch.from_numpy(dw.page_table).to(dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # 256 MB > L2
+    for _ in range(args.warmup):
+        st.run(p, W, vp, pt, stream)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.start()
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        st.run(p, W, vp, pt, stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    assert C.iamap_device_status(stream) == 0
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
+    ctx = int(dw.ctx_lens.sum())
+    byts = 2.0 * ctx * dw.H_r * dw.d_v + 4.0 * ctx * dw.H_s + 4.0 * dw.batch * dw.H_r * dw.d_v
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {
+        "metric": "decode rows/s (paged mapped_av, batch 4, context 8704)",
+        "value": round(dw.batch * world / (ms * 1e-3), 1), "unit": "rows/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": CONFIG_TEXT["decode"],
+                                        "l2": "256 MB flush between steps"},
+        "roofline": {"kernel": "paged_gemv", "bound": "hbm", "achieved": round(gbs, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "traffic": load_traffic("paged_gemv", ["decode.cu"])},
+        "clocks": clocks, "gpu_launches": 2 * args.steps,
+    }, dw
+
+
+def bench_headmatch(args, world, rank, local, peaks):
+    import torch
+    from synth import head_match_config
+    from cross_model_attention_map_b200 import iamap as C
+    from cross_model_attention_map_b200.runner import HeadMatch
+
+    dev = torch.device("cuda", local)
+    hm = head_match_config(seed=rank)
+    r = HeadMatch(hm.L_s, hm.H_small, hm.d_small, hm.L_l, hm.H_large, hm.d_large, hm.n,
+                  want_sim=False, device=dev)
+    qs, ks = bf16_dev(hm.q_small, dev), bf16_dev(hm.k_small, dev)
+    ql, kl = bf16_dev(hm.q_large, dev), bf16_dev(hm.k_large, dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        r.run(qs, ks, ql, kl, stream)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    barrier(world)
+    clk.start()
+    for a, b in evs:
+        a.record(stream)
+        r.run(qs, ks, ql, kl, stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    assert C.iamap_device_status(stream) == 0
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
+    nb = (hm.n + 63) // 64
+    K = nb * (nb + 1) // 2 * 4096
+    NS, NL = hm.L_s * hm.H_small, hm.L_l * hm.H_large
+    pairs = hm.n * (hm.n + 1) // 2
+    gram = 2.0 * NS * NL * pairs
+    maps = 2.0 * pairs * (NS * hm.d_small + NL * hm.d_large)
+    tf = (gram + maps) / (ms * 1e-3) / 1e12
+    return {
+        "metric": "head_match calibrations/s (n=1024, 336 small x 512 large heads)",
+        "value": round(world / (ms * 1e-3), 2), "unit": "calibrations/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": CONFIG_TEXT["headmatch"],
+                                        "gram_K_padded": K},
+        "roofline": {"kernel": "head_match (maps + gram)", "bound": "tensor",
+                     "achieved": round(tf, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None},
+        "clocks": clocks, "gpu_launches": 5 * args.steps,
+    }, hm
+
+
+def reference_arm(args):
+    """The float64 oracle on the host cores, same metric and unit, bounded sample per step."""
+    from synth import prefill_config
+    if args.config not in ("varlen40k", "prefill8k", "tiny"):
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "reference arm implemented for the prefill workloads only"}))
+        return
+    wl = prefill_config(args.config)
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample_prefill(wl, budget_s=budget, seed=99)
+    vals = []
+    text = ""
+    for i in range(args.steps):
+        v, rows, dt, text = oracle_sample_prefill(wl, budget_s=budget, seed=i)
+        vals.append(v)
+    value = statistics.mean(vals)
+    ms = 1e3 * sum(wl.seqlens) / value
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": CONFIG_TEXT[args.config]},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores(),
+                         "kind": "oracle", "sample": text + " per step"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="varlen40k", choices=sorted(CONFIG_TEXT))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        reference_arm(args)
+        return
+
+    world, rank, local = dist_setup(args)
+    peaks = load_peaks()
+    if args.config in ("varlen40k", "prefill8k", "tiny"):
+        line, wl = bench_prefill(args, world, rank, local, peaks)
+    elif args.config == "decode":
+        line, wl = bench_decode(args, world, rank, local, peaks)
+    else:
+        line, wl = bench_headmatch(args, world, rank, local, peaks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config in (
+            "varlen40k", "prefill8k", "tiny"):
+        v, rows, dt, text = oracle_sample_prefill(wl, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(v, 2), "unit": "tokens/s", "cores": cores(),
+                                "kind": "oracle", "sample": text + " in %.1f s" % dt}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
