@@ -57,6 +57,8 @@ _SIGS = {
     "iamap_mapped_av_paged_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "iamap_mapped_av_paged": (_I, [_P, _I, _P, _P, _I64, _P, _I, _I, _P, _P, _I, _I, _I, _I,
                                    _P, _P, _SZ, _P]),
+    "iamap_mapped_av_paged_noalloc": (_I, [_P, _I, _P, _P, _I64, _P, _I, _I, _P, _P, _I, _I, _I,
+                                           _I, _P, _P]),
     "iamap_head_match_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "iamap_head_match": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ,
                               _P]),
@@ -189,6 +191,18 @@ def iamap_mapped_av_paged(p_rows, ctx_stride, W, v_pages, num_pages, page_table,
         _ptr(p_rows), ctx_stride, _ptr(W), _ptr(v_pages), num_pages, _ptr(page_table), max_pages,
         page_size, _ptr(ctx_lens), cp, batch, H_s, H_r, d_v, _ptr(out), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def iamap_mapped_av_paged_noalloc(p_rows, ctx_stride, W, v_pages, num_pages, page_table,
+                                  max_pages, page_size, ctx_lens, ctx_lens_host, batch, H_s, H_r,
+                                  d_v, out, stream=None):
+    """The decode step without a workspace, for callers that cannot allocate device memory at
+    call time (the partial sums live in a fixed 16 MiB array inside the library)."""
+    cp, keep = _host_i32(ctx_lens_host)
+    _check("iamap_mapped_av_paged_noalloc", _lib.iamap_mapped_av_paged_noalloc(
+        _ptr(p_rows), ctx_stride, _ptr(W), _ptr(v_pages), num_pages, _ptr(page_table), max_pages,
+        page_size, _ptr(ctx_lens), cp, batch, H_s, H_r, d_v, _ptr(out), _stream(stream)))
     del keep
 
 

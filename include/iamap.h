@@ -177,6 +177,30 @@ int iamap_mapped_av_paged(const float* p_rows, int ctx_stride, const float* W,
                           float* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The paged decode step of iamap_mapped_av_paged for callers that cannot allocate device memory
+ * when they call: for example a serving engine that reserved nearly all GPU memory for its KV
+ * cache at start-up, or one that forbids cudaMalloc on its decode loop because cudaMalloc
+ * synchronises the device. The pages have no counterpart of this entry point; it exists only
+ * for such callers. Same arguments and result as iamap_mapped_av_paged, minus the workspace:
+ * the split partial sums live in a fixed 16 MiB device array inside the library, which every GPU
+ * that loads the library holds until the process exits. Nothing here allocates (no cudaMalloc,
+ * no cudaFree, no status word).
+ *   - The first call on a device looks up that array's device address and caches it; make that
+ *     first call before any stream capture.
+ *   - A call whose partial sums (batch x chunks x H_r x d_v floats) exceed 16 MiB returns
+ *     IAMAP_ERR_CAPACITY and launches nothing.
+ *   - All calls on a device share the array (it keeps the last call's contents; every value read
+ *     is first written by the same call). Calls that overlap on the GPU race on it: order them
+ *     on one stream.
+ *   - Out-of-range page indices are skipped and not reported (there is no status word).
+ */
+int iamap_mapped_av_paged_noalloc(const float* p_rows, int ctx_stride, const float* W,
+                                  const void* v_pages, int64_t num_pages,
+                                  const int32_t* page_table, int max_pages, int page_size,
+                                  const int32_t* ctx_lens, const int32_t* ctx_lens_host, int batch,
+                                  int H_s, int H_r, int d_v, float* out, void* stream);
+
+/*
  * Head matching (calibration). q_small / k_small bf16 [L_s, n, H_small, d_small];
  * q_large / k_large bf16 [L_l, n, H_large, d_large]. Each head's map is the causal softmax of
  * q k^T / sqrt(d) over the first n_used tokens (n_used <= n; the prompt truncation tau_t).
