@@ -13,7 +13,9 @@
 // Union index (row_count / row_scan / row_fill): the union of the heads' kept blocks per row
 // block, with head masks and tile offsets.
 // Stage 2 (compress_kernel<D, true>): recomputes each kept tile with the same arithmetic as
-// stage 1 and writes exp(s - lse) as a bf16 64 x 64 tile at its BSR position.
+// stage 1 and writes exp(s - lse) as bf16 at its BSR position. The k present heads of a stored
+// block are interleaved by row: row i of head rank t is at (i * k + t) * 64 within the block, so
+// one tile row of all present heads is a contiguous run (what mapped_av loads).
 #include "qk_tile.cuh"
 #include "internal.h"
 
@@ -55,8 +57,8 @@ static size_t stats_smem_bytes(int D, int max_nb) {
 static size_t extract_smem_bytes(int D, int max_nb) {
   return (size_t)2 * kTile * D * 2                       // key tiles (2 stages)
          + (size_t)kTile * kTile * 2                      // bf16 staging tile
-         + sizeof(int64_t) * (size_t)max_nb               // own tile indices
-         + sizeof(int) * (size_t)max_nb                   // own column blocks
+         + sizeof(int64_t) * (size_t)max_nb               // own block base tiles
+         + sizeof(int) * 2 * (size_t)max_nb               // own column blocks, (rank, k)
          + 16;                                            // own count
 }
 
@@ -211,9 +213,10 @@ __global__ void __launch_bounds__(kTileThreads) compress_kernel(CompressParams p
       if (sorted_s[rank_s[J]] < thr) atomicOr(hm_out + J, bit);
   } else {
     __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(rest);          // [64][64] swizzled
-    int64_t* own_tile = reinterpret_cast<int64_t*>(rest + kTile * kTile * 2);  // [max_nb]
-    int* own_J = reinterpret_cast<int*>(own_tile + p.max_nb);                // [max_nb]
-    int* own_cnt = own_J + p.max_nb;
+    int64_t* own_base = reinterpret_cast<int64_t*>(rest + kTile * kTile * 2);  // [max_nb]
+    int* own_J = reinterpret_cast<int*>(own_base + p.max_nb);                // [max_nb]
+    int* own_rk = own_J + p.max_nb;                                           // rank | k << 8
+    int* own_cnt = own_rk + p.max_nb;
     // The column blocks this head keeps in this row block, with their tile indices.
     if (warp == 0) {
       const int u0 = p.row_ptr[rb], u1 = p.row_ptr[rb + 1];
@@ -231,7 +234,8 @@ __global__ void __launch_bounds__(kTileThreads) compress_kernel(CompressParams p
         if (own) {
           const int pos = cnt + __popc(b & ((1u << lane) - 1u));
           own_J[pos] = p.col_idx[u];
-          own_tile[pos] = p.val_off[u] + __popcll(m & below);
+          own_base[pos] = p.val_off[u];
+          own_rk[pos] = __popcll(m & below) | (__popcll(m) << 8);
         }
         cnt += __popc(b);
       }
@@ -270,13 +274,15 @@ __global__ void __launch_bounds__(kTileThreads) compress_kernel(CompressParams p
             pack_bf16(p2, p3);
       }
       __syncthreads();
-      const int64_t tile = own_tile[t];
-      if (tile >= 0 && tile < p.capacity) {
-        uint4* dst = reinterpret_cast<uint4*>(p.vals + tile * (kTile * kTile));
+      const int64_t base = own_base[t];
+      const int rank = own_rk[t] & 255, kk = own_rk[t] >> 8;
+      if (base >= 0 && base + kk <= p.capacity) {
+        __nv_bfloat16* blk = p.vals + base * (kTile * kTile) + (int64_t)rank * kTile;
 #pragma unroll
         for (int c = tid; c < kTile * 8; c += kTileThreads) {
           const int r = c >> 3, ch = c & 7;
-          dst[c] = *reinterpret_cast<const uint4*>(stage + r * kTile + ((ch ^ (r & 7)) << 3));
+          *reinterpret_cast<uint4*>(blk + (int64_t)r * kk * kTile + ch * 8) =
+              *reinterpret_cast<const uint4*>(stage + r * kTile + ((ch ^ (r & 7)) << 3));
         }
       } else {
         cap_flag = true;

@@ -64,6 +64,9 @@ struct MappedAvArgs {
   unsigned int* status = nullptr;
 };
 int mapped_av_impl(const MappedAvArgs& a, cudaStream_t stream);
+// Tensor-core, cluster-cooperative form (mapped_av_tc.cu); used when supported.
+bool mapped_av_tc_supported(int H_s, int H_r, int d_v);
+int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream);
 
 struct PagedArgs {
   const float* p_rows = nullptr;

@@ -12,6 +12,8 @@
 //   3. warp w computes O_r[16 rows] += P_r . V_r[J] with mma.sync (bf16 in, fp32 accumulate)
 //      for receiver head r = w / 4 of the group, V_r[J] staged in shared memory.
 // The output rows are written once, after the last column block.
+// This form serves receiver layers wider than the tensor-core kernel's cluster (H_r > 32); the
+// tensor-core, cluster-cooperative kernel (mapped_av_tc.cu) handles H_r <= 32.
 #include "internal.h"
 
 namespace iamap {
@@ -119,10 +121,12 @@ __global__ void __launch_bounds__(kAvThreads, 1) mapped_av_kernel(AvParams p) {
       for (int e = tid; e < kAvChunk * kTileElems / 8; e += kAvThreads) {
         const int t = e / (kTileElems / 8), off = e % (kTileElems / 8);
         const int hr = c * kAvChunk + t;
-        const int64_t tile = base + hr;
-        const bool valid = hr < k && tile >= 0 && tile < p.capacity;
+        const bool valid = hr < k && base >= 0 && base + k <= p.capacity;
         if (hr < k && !valid) bad_index = true;
-        const __nv_bfloat16* src = p.vals + (valid ? tile * kTileElems + off * 8 : 0);
+        // row i of head rank hr: (i * k + hr) * 64 elements into the block
+        const int i = off >> 3, ch = off & 7;
+        const __nv_bfloat16* src =
+            p.vals + (valid ? base * kTileElems + ((int64_t)i * k + hr) * kT + ch * 8 : 0);
         cp_async16(smem_u32(sT + (buf * kAvChunk + t) * kTileElems + off * 8), src, valid);
       }
     };
@@ -232,6 +236,7 @@ static int launch_av(const AvParams& p, int64_t num_items, cudaStream_t stream) 
 }
 
 int mapped_av_impl(const MappedAvArgs& a, cudaStream_t stream) {
+  if (mapped_av_tc_supported(a.H_s, a.H_r, a.d_v)) return mapped_av_tc_impl(a, stream);
   AvParams p{};
   p.cu = a.cu_seqlens;
   p.tab = a.tab;

@@ -1,0 +1,486 @@
+// mapped_av on the 5th-generation tensor cores, one thread-block cluster per row block.
+//
+// What it computes is the fused mapping + value aggregation of the MapFlow news page ("PKU
+// MapFlow: cross-model attention map reuse", storage-and-execution part, third component): for
+// every stored block (I, J) of the block-sparse sender map, P_r = sum_s W[r, s] Pt_s is formed on
+// chip and O_r[rows of I] += P_r . V_r[rows of J]; no dense receiver map exists anywhere.
+//
+// Work split. A CTA can keep O accumulators of 4 receiver heads x 64 rows x d_v in TMEM, so a row
+// block needs C = ceil(H_r / 4) CTAs; they form one cluster and split the sender tiles instead of
+// each reading all of them:
+//   * CTA c TMA-loads rows [2*c0, 2*c1) of every present sender tile of the block. The values of
+//     a stored block are interleaved by row (row i of head rank t at line i*k + t), so one tile
+//     row of all k present heads is one contiguous run of k lines of 128 B: one box per row,
+//     whose lines are the K-stack of an MN-major, 128-byte-swizzled operand. It mixes them for ALL receiver
+//     heads: D[128 positions][N = H_r] = P[128][K = heads] . W'[N][K] with tcgen05.mma, where W'
+//     holds the W columns of the present heads (zero past them).
+//   * The mixed rows are rounded to bf16, transposed through a 2 KB per-warp scratch into 16-byte
+//     runs of 8 positions of one receiver head, and stored with st.async straight into the receive
+//     buffer of the CTA owning that head, at their place in its K-major, 128-byte-swizzled tile;
+//     the bytes count on that CTA's mbarrier.
+//   * Each CTA accumulates O_r^T[d_v][64 rows] += V_r[J]^T . P_r^T for its 4 heads: V_r[J] is the
+//     MN-major A operand (TMA), the received P_r the K-major B operand; accumulators stay in TMEM
+//     across the whole row and are written once.
+// No TMA multicast is used: every CTA loads its own tiles.
+//
+// Roles: warp 0 loads the sender slices, warp 7 builds W', warp 6 loads the V tiles, one thread of
+// warp 1 issues every tcgen05.mma (mixing of block t+1 before P.V of block t, so the exchange of
+// block t overlaps the next mixing), warps 2-5 read the mixing results out of TMEM, stage and send
+// them, and write the output. Every wait is bounded (2 s, then IAMAP_DEV_TIMEOUT).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+#include "tc_utils.cuh"
+
+namespace iamap {
+
+// ------------------------------------------------------------------------------------------------
+// Tensor-map encoding through the runtime's driver entry point
+// ------------------------------------------------------------------------------------------------
+
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::once_flag g_encode_once;
+
+int encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return set_error(IAMAP_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return set_error(IAMAP_ERR_INVALID_ARG, "tensor map encoding failed (%d)", (int)r);
+  return IAMAP_OK;
+}
+
+namespace tcav {
+
+constexpr int kG = 4;            // receiver heads per CTA (O in TMEM: 4 x 64 columns)
+constexpr int kNP = 6;           // sender-slice ring (1.5 blocks of slices at C = 8)
+constexpr int kND = 4;           // mixing-result TMEM slots
+constexpr int kNV = 4;           // V-tile ring (one block's worth for 4 heads)
+constexpr int kThreads = 256;    // 8 warps
+constexpr int kMixCol = 256;     // first TMEM column of the mixing slots
+constexpr uint32_t kTmemCols = 512;
+
+// barrier indices
+enum {
+  P_FULL = 0, P_EMPTY = P_FULL + kNP, W_FULL = P_EMPTY + kNP, W_EMPTY = W_FULL + 2,
+  D_FULL = W_EMPTY + 2, D_EMPTY = D_FULL + kND, RECV_FULL = D_EMPTY + kND, BUF_FREE = RECV_FULL + 2,
+  V_FULL = BUF_FREE + 2, V_EMPTY = V_FULL + kNV, O_FULL = V_EMPTY + kNV, NUM_BARS = O_FULL + 1
+};
+
+struct __align__(64) Params {
+  CUtensorMap p_maps[8];   // BSR values viewed [capacity * 64 lines][64]; box {64, 8 * (i + 1)}
+  CUtensorMap v_map;       // V viewed [n][H_r * d_v]; box {64, 64}
+  const int32_t* cu;
+  SeqTables tab;
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  const unsigned long long* headmask;
+  const int64_t* val_off;
+  const float* W;
+  float* out;
+  unsigned int* status;
+  int H_s, H_r, d_v, C, NR, KH, RB;
+  uint32_t off_p, off_w, off_scr, off_recv, off_v, off_wf, off_bar;
+};
+
+__device__ __forceinline__ uint32_t bar_addr(uint32_t base, int i) { return base + 8u * (uint32_t)i; }
+
+__global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_constant__ Params p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + p.off_bar;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + p.off_bar + 8 * NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int C = p.C;
+  const uint32_t crank = tc::cluster_rank();
+  const int item = blockIdx.x / C;
+  const int2 it = p.tab.items[item];
+  const int s = it.x, I = it.y;
+  const int seq0 = p.cu[s];
+  const int L = p.cu[s + 1] - seq0;
+  const int rb = p.tab.rb_start[s] + I;
+  const int u0 = p.row_ptr[rb];
+  const int T = p.row_ptr[rb + 1] - u0;
+  const int r0 = (int)crank * kG;
+  const int G = max(0, min(kG, p.H_r - r0));
+  const int c0 = (32 * (int)crank) / C, c1 = (32 * ((int)crank + 1)) / C;
+  const uint32_t p_box = (uint32_t)p.RB * 128u;   // one box: RB lines of 128 B
+  const uint32_t p_stage = 2u * p_box;
+  const uint32_t w_stage = (uint32_t)p.NR * 128u;
+  const uint32_t v_stage = (uint32_t)p.d_v * 128u;
+
+  // ---- set-up: barriers, zeroed sender ring and its 1 KB tail (lines the MMA reads past a box
+  // must be finite: their weights are zero), W, TMEM ----
+  if (tid == 0) {
+    for (int i = 0; i < NUM_BARS; ++i) {
+      uint32_t cnt = 1;
+      if (i >= D_EMPTY && i < D_EMPTY + kND) cnt = 4;
+      if (i >= BUF_FREE && i < BUF_FREE + 2) cnt = (uint32_t)C;
+      tc::mbar_init(bar_addr(bars, i), cnt);
+    }
+    misc[1] = 0;
+    tc::fence_barrier_init();
+  }
+  {
+    uint4* z = reinterpret_cast<uint4*>(smem + p.off_p);
+    const int nz = (int)((kNP * p_stage + 1024u) / 16);
+    for (int i = tid; i < nz; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
+    float* wf = reinterpret_cast<float*>(smem + p.off_wf);   // W transposed: [H_s][H_r]
+    for (int i = tid; i < p.H_r * p.H_s; i += kThreads) {
+      const int r = i / p.H_s, h = i - r * p.H_s;
+      wf[h * p.H_r + r] = p.W[i];
+    }
+    tc::fence_proxy_async_smem();
+  }
+  if (warp == 1) tc::tmem_alloc(smem_u32(misc), kTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  tc::cluster_sync();  // every CTA's barriers exist before any remote copy or arrival
+  const uint32_t tmem = misc[0];
+
+  if (warp == 0) {
+    // ------------------------------ sender slices ------------------------------
+    if (lane == 0) {
+      int q = 0;
+      unsigned long long m_next = T > 0 ? p.headmask[u0] : 0ull;
+      int64_t off_next = T > 0 ? p.val_off[u0] : 0;
+      for (int t = 0; t < T; ++t) {
+        const unsigned long long m = m_next;
+        const int64_t off = off_next;
+        if (t + 1 < T) {
+          m_next = p.headmask[u0 + t + 1];
+          off_next = p.val_off[u0 + t + 1];
+        }
+        const int k = __popcll(m);
+        const int k8 = (k + 7) >> 3;
+        const int y0 = (int)(off * 64);   // first line of the block
+        for (int ch = c0; ch < c1; ++ch, ++q) {
+          const int ps = q % kNP;
+          if (q >= kNP) tc::wait_bar(bar_addr(bars, P_EMPTY + ps), ((q / kNP) - 1) & 1, abort_flag, p.status);
+          const uint32_t dst = sbase + p.off_p + ps * p_stage;
+          tc::mbar_expect_tx(bar_addr(bars, P_FULL + ps), 2u * (uint32_t)k8 * 8u * 128u);
+          tc::tma_load_2d(dst, &p.p_maps[k8 - 1], 0, y0 + (2 * ch) * k, bar_addr(bars, P_FULL + ps));
+          tc::tma_load_2d(dst + p_box, &p.p_maps[k8 - 1], 0, y0 + (2 * ch + 1) * k,
+                          bar_addr(bars, P_FULL + ps));
+        }
+      }
+    }
+  } else if (warp == 7) {
+    // ------------------------------ W' of each stored block ------------------------------
+    // row r = receiver head r; column t = W[r][t-th present sender head]; zero past k and for
+    // padding rows. The present-head list comes from two ballots.
+    const float* wf = reinterpret_cast<const float*>(smem + p.off_wf);
+    unsigned char* hl = smem + p.off_bar + 8 * NUM_BARS + 16;   // 64-byte head list
+    unsigned long long m_next = T > 0 ? p.headmask[u0] : 0ull;
+    for (int t = 0; t < T; ++t) {
+      const unsigned long long m = m_next;
+      if (t + 1 < T) m_next = p.headmask[u0 + t + 1];
+      const int k = __popcll(m);
+      const int ws = t & 1;
+      if (t >= 2) tc::wait_bar(bar_addr(bars, W_EMPTY + ws), ((t - 2) >> 1) & 1, abort_flag, p.status);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int h = 32 * half + lane;
+        const bool present = (m >> h) & 1ull;
+        const unsigned b = __ballot_sync(0xffffffffu, present);
+        const int base = half ? __popcll(m & 0xffffffffull) : 0;
+        if (present) hl[base + __popc(b & ((1u << lane) - 1u))] = (unsigned char)h;
+      }
+      __syncwarp();
+      if (lane < p.NR) {
+        const int r = lane;
+        unsigned char* row = smem + p.off_w + ws * w_stage + r * 128;
+        const bool real = r < p.H_r;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int tt = 8 * c + e;
+            f[e] = (real && tt < k) ? wf[hl[tt] * p.H_r + r] : 0.f;
+          }
+          uint4 pk;
+          pk.x = pack_bf16(f[0], f[1]);
+          pk.y = pack_bf16(f[2], f[3]);
+          pk.z = pack_bf16(f[4], f[5]);
+          pk.w = pack_bf16(f[6], f[7]);
+          *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = pk;
+        }
+      }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_addr(bars, W_FULL + ws));
+      __syncwarp();
+    }
+  } else if (warp == 6) {
+    // ------------------------------ V tiles ------------------------------
+    if (lane == 0) {
+      int vq = 0;
+      int J_next = T > 0 ? p.col_idx[u0] : 0;
+      for (int t = 0; t < T; ++t) {
+        const int J = J_next;
+        if (t + 1 < T) J_next = p.col_idx[u0 + t + 1];
+        for (int rl = 0; rl < G; ++rl, ++vq) {
+          const int vs = vq % kNV;
+          if (vq >= kNV) tc::wait_bar(bar_addr(bars, V_EMPTY + vs), ((vq / kNV) - 1) & 1, abort_flag, p.status);
+          const uint32_t dst = sbase + p.off_v + vs * v_stage;
+          tc::mbar_expect_tx(bar_addr(bars, V_FULL + vs), v_stage);
+          const int x = (r0 + rl) * p.d_v, y = seq0 + J * 64;
+          tc::tma_load_2d(dst, &p.v_map, x, y, bar_addr(bars, V_FULL + vs));
+          if (p.d_v == 128) tc::tma_load_2d(dst + 8192u, &p.v_map, x + 64, y, bar_addr(bars, V_FULL + vs));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issue ------------------------------
+    if (lane == 0) {
+      const uint32_t id_mix = tc::idesc_bf16(128, p.NR, 1, 0);
+      const uint32_t id_pv = tc::idesc_bf16(128, 64, 1, 0);
+      const uint32_t v_lbo = p.d_v == 128 ? 8192u : 0u;
+      const uint16_t all_ctas = (uint16_t)((1u << C) - 1u);
+      int q = 0, vq = 0;
+      auto pv = [&](int t) {
+        const int rs = t & 1;
+        tc::mbar_expect_tx(bar_addr(bars, RECV_FULL + rs), (uint32_t)G * 8192u);
+        tc::wait_bar(bar_addr(bars, RECV_FULL + rs), (t >> 1) & 1, abort_flag, p.status);
+        tc::tc_fence_after();
+        tc::fence_proxy_async_smem();  // peers' st.async data, read next by the tensor cores
+        for (int rl = 0; rl < G; ++rl, ++vq) {
+          const int vs = vq % kNV;
+          tc::wait_bar(bar_addr(bars, V_FULL + vs), (vq / kNV) & 1, abort_flag, p.status);
+          tc::tc_fence_after();
+          const uint32_t va = sbase + p.off_v + vs * v_stage;
+          const uint32_t pb = sbase + p.off_recv + (uint32_t)rs * (kG * 8192u) + (uint32_t)rl * 8192u;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t a = tc::sdesc_sw128(va + kk * 2048u, v_lbo, 1024u);
+            const uint64_t b = tc::sdesc_sw128(pb + kk * 32u, 16u, 1024u);
+            tc::mma_bf16(tmem + (uint32_t)rl * 64u, a, b, id_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::mma_commit(bar_addr(bars, V_EMPTY + vs));
+        }
+        tc::mma_commit_to_cluster(bar_addr(bars, BUF_FREE + rs), all_ctas);
+      };
+      int k_next = T > 0 ? __popcll(p.headmask[u0]) : 0;
+      for (int t = 0; t < T; ++t) {
+        const int ksteps = (k_next + 15) >> 4;
+        if (t + 1 < T) k_next = __popcll(p.headmask[u0 + t + 1]);
+        const int ws = t & 1;
+        tc::wait_bar(bar_addr(bars, W_FULL + ws), (t >> 1) & 1, abort_flag, p.status);
+        tc::tc_fence_after();
+        const uint32_t wb = sbase + p.off_w + ws * w_stage;
+        for (int ch = c0; ch < c1; ++ch, ++q) {
+          const int ps = q % kNP, ds = q % kND;
+          tc::wait_bar(bar_addr(bars, P_FULL + ps), (q / kNP) & 1, abort_flag, p.status);
+          if (q >= kND) tc::wait_bar(bar_addr(bars, D_EMPTY + ds), ((q / kND) - 1) & 1, abort_flag, p.status);
+          tc::tc_fence_after();
+          const uint32_t pa = sbase + p.off_p + ps * p_stage;
+          const uint32_t d = tmem + (uint32_t)kMixCol + (uint32_t)ds * (uint32_t)p.NR;
+          for (int kk = 0; kk < ksteps; ++kk) {
+            const uint64_t a = tc::sdesc_sw128(pa + kk * 2048u, p_box, 1024u);
+            const uint64_t b = tc::sdesc_sw128(wb + kk * 32u, 16u, 1024u);
+            tc::mma_bf16(d, a, b, id_mix, kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(bar_addr(bars, P_EMPTY + ps));
+          tc::mma_commit(bar_addr(bars, D_FULL + ds));
+        }
+        tc::mma_commit(bar_addr(bars, W_EMPTY + ws));
+        if (t > 0) pv(t - 1);
+      }
+      if (T > 0) pv(T - 1);
+      tc::mma_commit(bar_addr(bars, O_FULL));
+    }
+  } else {
+    // ------------------------------ readout, exchange, output (warps 2-5) ------------------------------
+    const int e = warp & 3;               // TMEM lane quarter of this warp
+    const uint32_t lane_base = (uint32_t)(32 * e) << 16;
+    unsigned char* scr = smem + p.off_scr + (warp - 2) * 2048;   // [32 heads][32 positions] bf16
+    const int o = lane & 3;               // this lane's 16-byte run: positions 8*o .. 8*o+7
+    const int rq = lane >> 2;             // this lane's heads: 8*v + rq
+    int q = 0;
+    for (int t = 0; t < T; ++t) {
+      const int ss = t & 1;
+      // the receive buffers of round t-2 are free once every peer's P.V of that round completed
+      if (t >= 2) tc::wait_bar(bar_addr(bars, BUF_FREE + ss), ((t - 2) >> 1) & 1, abort_flag, p.status);
+      const uint32_t recv_local = sbase + p.off_recv + (uint32_t)ss * (kG * 8192u);
+      const uint32_t rbar_local = bar_addr(bars, RECV_FULL + ss);
+      for (int ch = c0; ch < c1; ++ch, ++q) {
+        const int ds = q % kND;
+        tc::wait_bar(bar_addr(bars, D_FULL + ds), (q / kND) & 1, abort_flag, p.status);
+        tc::tc_fence_after();
+        uint32_t v[32];
+        const uint32_t ta = tmem + lane_base + (uint32_t)kMixCol + (uint32_t)ds * (uint32_t)p.NR;
+        if (p.NR == 32) {
+          IAMAP_TMEM_LD32(ta, v);
+        } else {
+          IAMAP_TMEM_LD16(ta, v);
+#pragma unroll
+          for (int i = 16; i < 32; ++i) v[i] = 0u;
+        }
+        tc::tmem_ld_wait();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar_addr(bars, D_EMPTY + ds));
+        // transpose: position = lane, head = register  ->  16-byte runs of one head
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+          if (r < p.NR)
+            reinterpret_cast<__nv_bfloat16*>(scr)[r * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[r]));
+        __syncwarp();
+        const int pos0 = 32 * e;                          // this warp's first position in the chunk
+        const int arow = 2 * ch + (pos0 >> 6);            // tile row
+        const int jc = ((pos0 & 63) >> 3) + o;            // 16-byte chunk of the row
+        const uint32_t row_off = (uint32_t)arow * 128u + ((uint32_t)(jc ^ (arow & 7)) << 4);
+#pragma unroll
+        for (int vv = 0; vv < 4; ++vv) {
+          const int r = 8 * vv + rq;
+          if (r < p.H_r) {
+            const uint4 val = *reinterpret_cast<const uint4*>(scr + r * 64 + o * 16);
+            const uint32_t c2 = (uint32_t)(r >> 2);
+            const uint32_t dst = tc::map_to_cta(recv_local + (uint32_t)(r & 3) * 8192u + row_off, c2);
+            tc::st_async_v4(dst, val, tc::map_to_cta(rbar_local, c2));
+          }
+        }
+        __syncwarp();
+      }
+    }
+    // output rows: TMEM lane = d_v index, column = rl * 64 + row of the block
+    tc::wait_bar(bar_addr(bars, O_FULL), 0, abort_flag, p.status);
+    tc::tc_fence_after();
+    const int dv = 32 * e + lane;
+    if (32 * e < p.d_v) {
+      for (int rl = 0; rl < G; ++rl) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
+          IAMAP_TMEM_LD32(tmem + lane_base + (uint32_t)(rl * 64 + half * 32), v);
+          tc::tmem_ld_wait();
+          float* o = p.out + ((int64_t)(seq0 + I * 64 + half * 32) * p.H_r + r0 + rl) * p.d_v + dv;
+#pragma unroll
+          for (int ii = 0; ii < 32; ++ii)
+            if (I * 64 + half * 32 + ii < L)
+              o[(int64_t)ii * p.H_r * p.d_v] = T > 0 ? __uint_as_float(v[ii]) : 0.f;
+        }
+      }
+    }
+    // the last two exchange rounds: every peer has consumed this CTA's copies and arrived here
+    for (int t = max(0, T - 2); t < T; ++t)
+      tc::wait_bar(bar_addr(bars, BUF_FREE + (t & 1)), (t >> 1) & 1, abort_flag, p.status);
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+  tc::cluster_sync();
+}
+
+}  // namespace tcav
+
+static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool mapped_av_tc_supported(int H_s, int H_r, int d_v) {
+  return H_s >= 1 && H_s <= 64 && H_r >= 1 && H_r <= 32 && (d_v == 64 || d_v == 128);
+}
+
+int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream) {
+  using namespace tcav;
+  Params p{};
+  const int C = (a.H_r + kG - 1) / kG;
+  p.C = C;
+  p.H_s = a.H_s;
+  p.H_r = a.H_r;
+  p.d_v = a.d_v;
+  p.NR = a.H_r <= 16 ? 16 : 32;
+  p.KH = (a.H_s + 15) / 16 * 16;
+  p.RB = (a.H_s + 7) / 8 * 8;
+  size_t off = 0;
+  p.off_p = (uint32_t)off;
+  off += (size_t)kNP * 2 * p.RB * 128 + 1024;   // ring + tail read past the last box
+  off = round_up(off, 1024);
+  p.off_w = (uint32_t)off;
+  off += (size_t)2 * p.NR * 128;
+  off = round_up(off, 1024);
+  p.off_recv = (uint32_t)off;
+  off += (size_t)2 * kG * 8192;
+  p.off_v = (uint32_t)off;
+  off += (size_t)kNV * a.d_v * 128;
+  p.off_scr = (uint32_t)off;
+  off += (size_t)4 * 2048;
+  p.off_wf = (uint32_t)off;
+  off += sizeof(float) * (size_t)a.H_r * a.H_s;
+  off = round_up(off, 8);
+  p.off_bar = (uint32_t)off;
+  off += 8 * NUM_BARS + 16 + 64;   // barriers, TMEM address + abort flag, head list
+  const size_t smem = off + 1024;  // alignment slack
+  if (smem > 232448)
+    return set_error(IAMAP_ERR_UNSUPPORTED, "mapped_av needs %zu bytes of shared memory", smem);
+
+  const uint64_t cap = (uint64_t)std::max<int64_t>(a.capacity, 1);
+  for (int i = 0; i < 8; ++i) {
+    int rc = encode_tmap_2d_bf16(&p.p_maps[i], a.vals, 64, cap * 64, 128, 64, (uint32_t)(8 * (i + 1)));
+    if (rc) return rc;
+  }
+  int rc = encode_tmap_2d_bf16(&p.v_map, a.v, (uint64_t)a.H_r * a.d_v, (uint64_t)a.n,
+                               (uint64_t)a.H_r * a.d_v * 2, 64, 64);
+  if (rc) return rc;
+  p.cu = a.cu_seqlens;
+  p.tab = a.tab;
+  p.row_ptr = a.row_ptr;
+  p.col_idx = a.col_idx;
+  p.headmask = reinterpret_cast<const unsigned long long*>(a.headmask);
+  p.val_off = a.val_off;
+  p.W = a.W;
+  p.out = a.out;
+  p.status = a.status;
+
+  IAMAP_CUDA_CHECK(cudaFuncSetAttribute(mapped_av_tc_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (a.plan.num_rowblocks == 0) return IAMAP_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.plan.num_rowblocks * C), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  IAMAP_CUDA_CHECK(cudaOccupancyMaxActiveClusters(&clusters, mapped_av_tc_kernel, &cfg));
+  if (clusters < 1)
+    return set_error(IAMAP_ERR_UNSUPPORTED, "a cluster of %d CTAs with %zu bytes each cannot be "
+                     "scheduled", C, smem);
+  IAMAP_CUDA_CHECK(cudaLaunchKernelEx(&cfg, mapped_av_tc_kernel, p));
+  return IAMAP_OK;
+}
+
+}  // namespace iamap

@@ -47,10 +47,12 @@
  *     row_ptr  int32 [num_rowblocks + 1]
  *     col_idx  int32 [nnz_blocks]   column-block index J (local to the sequence)
  *     headmask u64   [nnz_blocks]   present sender heads
- *     val_off  int64 [nnz_blocks]   tile index of the first present head; the tiles of the
- *                                   present heads follow in increasing head order
- *     vals     bf16  [tiles, B, B]  row-major probability tiles; causally masked entries and rows
- *                                   past the sequence end are 0
+ *     val_off  int64 [nnz_blocks]   first tile of the block; a block with k present heads
+ *                                   occupies tiles [val_off, val_off + k)
+ *     vals     bf16  [tiles, B, B]  probabilities, interleaved by row within a block: row i of the
+ *                                   head of rank t (t-th present head in increasing order) is at
+ *                                   element (val_off*B + i*k + t) * B; causally masked entries and
+ *                                   rows past the sequence end are 0
  *   out       fp32 [n, H_r, d_v]
  */
 #ifndef IAMAP_H
@@ -124,7 +126,7 @@ int iamap_compress_stats(const void* q, const void* k, const int32_t* cu_seqlens
 /*
  * Compress, stage 2 (extraction of the kept blocks). Recomputes each kept (head, row block,
  * column block) tile of probabilities exp(s_ij - lse_i) from q, k and stage 1's lse, and writes
- * it as a bf16 B x B tile at its BSR position. A tile whose index is >= vals_capacity_tiles is not
+ * it as bf16 at its BSR position (row-interleaved within the block, see Layouts). A tile whose index is >= vals_capacity_tiles is not
  * written and sets IAMAP_DEV_CAPACITY in the device status. After the last tile the call also
  * zero-fills up to 64 further tiles that fit in the capacity (mapped_av may read that far).
  */

@@ -62,6 +62,13 @@ def bsr_readback(layer):
     return row_ptr, col_idx, headmask, val_off, tiles
 
 
+def head_tile(vals, val_off_u, k, rank):
+    """[64, 64] tile of head rank `rank` in a stored block of k present heads: the block's values
+    are interleaved by row, row i of rank t at line i * k + t."""
+    blk = vals[int(val_off_u) * 64:(int(val_off_u) + k) * 64]
+    return blk.reshape(64, k, 64)[:, rank, :]
+
+
 def check_bsr_structure(layer, kept_gpu, lay):
     """The union index the GPU wrote equals the union of its own per-head kept sets."""
     row_ptr, col_idx, headmask, val_off, tiles = bsr_readback(layer)

@@ -16,7 +16,7 @@ import oracle as O
 from synth import bf16_bits_to_f64, make_prefill, prefill_config
 
 from _gpu_common import (LSE_ATOL, MASS_NORM_ATOL, bsr_readback, check_bsr_structure,
-                         check_output, compare_kept, gpu_kept, upload_prefill)
+                         check_output, compare_kept, gpu_kept, head_tile, upload_prefill)
 
 pytestmark = pytest.mark.gpu
 
@@ -59,7 +59,7 @@ def _full_parity(C, wl):
     flips = compare_kept(kept, ref.kept, ref.near)
     # BSR index from the GPU's own kept sets, and every stored tile
     row_ptr, col_idx, headmask, val_off = check_bsr_structure(layer, kept, lay)
-    vals = layer.vals.float().cpu().numpy()
+    vals = layer.vals.float().cpu().numpy().reshape(-1, 64)
     rb = 0
     for s in range(len(lay.seqlens)):
         for I in range(lay.nb[s]):
@@ -74,7 +74,7 @@ def _full_parity(C, wl):
                             stats[h] = O.rowblock_stats(wl.q, wl.k, wl.cu_seqlens, s, h, I, wl.B,
                                                         wl.tau, wl.bias_window, wl.bias_value)
                         t_ref = O.masked_tile(stats[h], J, wl.B)
-                        t_gpu = vals[val_off[u] + rank]
+                        t_gpu = head_tile(vals, val_off[u], bin(m).count("1"), rank)
                         np.testing.assert_allclose(t_gpu, t_ref, rtol=8e-3, atol=2e-6)
                         rank += 1
             rb += 1
@@ -162,7 +162,7 @@ def _sampled_parity(C, wl, samples):
     lse = layer.bufs["lse"].cpu().numpy()
     mass = layer.bufs["mass"].cpu().numpy()
     row_ptr, col_idx, headmask, val_off, tiles = bsr_readback(layer)
-    vals = layer.vals
+    vals = layer.vals.view(-1, 64)
     out = layer.out.cpu().numpy()
     flips = 0
     # invariants everywhere: kept normalised mass >= tau (up to fp32 rounding) per (head, block)
@@ -189,7 +189,9 @@ def _sampled_parity(C, wl, samples):
             rank = 0
             for h in range(wl.H_s):
                 if (m >> h) & 1:
-                    t_gpu = vals[val_off[u] + rank].float().cpu().numpy()
+                    k = bin(m).count("1")
+                    blk = vals[int(val_off[u]) * 64:(int(val_off[u]) + k) * 64].float().cpu().numpy()
+                    t_gpu = blk.reshape(64, k, 64)[:, rank, :]
                     np.testing.assert_allclose(t_gpu, O.masked_tile(st[h], J, wl.B), rtol=8e-3,
                                                atol=2e-6)
                     rank += 1
