@@ -23,10 +23,10 @@
 //     across the whole row and are written once.
 // No TMA multicast is used: every CTA loads its own tiles.
 //
-// Roles: warp 0 loads the sender slices, warp 7 builds W', warp 6 loads the V tiles, one thread of
-// warp 1 issues every tcgen05.mma (mixing of block t+1 before P.V of block t, so the exchange of
-// block t overlaps the next mixing), warps 2-5 read the mixing results out of TMEM, stage and send
-// them, and write the output. Every wait is bounded (2 s, then IAMAP_DEV_TIMEOUT).
+// Roles: warps 0, 8, 9, 10 load the sender slices, warp 7 builds W', warps 6 and 11 load the V
+// tiles, one thread of warp 1 issues the mixing MMAs and one thread of warp 12 the P.V MMAs (two
+// issuers: MMA and commit issue costs add up on one thread), warps 2-5 read the mixing results
+// out of TMEM, transpose and send them, and write the output. Every wait is bounded (2 s, then IAMAP_DEV_TIMEOUT).
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -68,26 +68,59 @@ int encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint
   return IAMAP_OK;
 }
 
+int encode_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                        uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                        uint32_t b2) {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return set_error(IAMAP_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return set_error(IAMAP_ERR_INVALID_ARG, "3-D tensor map encoding failed (%d)", (int)r);
+  return IAMAP_OK;
+}
+
 namespace tcav {
 
 constexpr int kG = 4;            // receiver heads per CTA (O in TMEM: 4 x 64 columns)
-constexpr int kNP = 6;           // sender-slice ring (1.5 blocks of slices at C = 8)
-constexpr int kND = 4;           // mixing-result TMEM slots
-constexpr int kNV = 4;           // V-tile ring (one block's worth for 4 heads)
-constexpr int kThreads = 256;    // 8 warps
+constexpr int kMaxNP = 12;       // sender-slice ring: as many slots as shared memory allows
+// One warp issues TMA loads at only ~3 M per second (about 25 GB/s of 8 KB boxes, measured on
+// this B200 whatever the box layout), so the loads are spread over several producer warps: four
+// for the sender slices (chunks round-robin), two for the V tiles (receiver heads alternating),
+// and each V tile (both 64-dim halves of one head) is a single 3-D box.
+constexpr int kPWarps = 4, kVWarps = 2;
+constexpr int kND = 8;           // mixing-result TMEM slots (chunks)
+constexpr int kNG = kND / 2;     // ... committed and released in pairs of chunks (one commit costs
+                                 // ~90 ns of issue time on this B200, an MMA ~25 ns)
+constexpr int kNV = 4;           // V tiles: one slot per receiver head of the CTA
+constexpr int kThreads = 416;    // 13 warps
 constexpr int kMixCol = 256;     // first TMEM column of the mixing slots
 constexpr uint32_t kTmemCols = 512;
 
 // barrier indices
 enum {
-  P_FULL = 0, P_EMPTY = P_FULL + kNP, W_FULL = P_EMPTY + kNP, W_EMPTY = W_FULL + 2,
-  D_FULL = W_EMPTY + 2, D_EMPTY = D_FULL + kND, RECV_FULL = D_EMPTY + kND, BUF_FREE = RECV_FULL + 2,
-  V_FULL = BUF_FREE + 2, V_EMPTY = V_FULL + kNV, O_FULL = V_EMPTY + kNV, NUM_BARS = O_FULL + 1
+  P_FULL = 0, P_EMPTY = P_FULL + kMaxNP, W_FULL = P_EMPTY + kMaxNP, W_EMPTY = W_FULL + 2,
+  D_FULL = W_EMPTY + 2, D_EMPTY = D_FULL + kNG, RECV_FULL = D_EMPTY + kNG, BUF_FREE = RECV_FULL + 2,
+  V_FULL = BUF_FREE + 2, PV_DONE = V_FULL + kNV, O_FULL = PV_DONE + 2, MIX_DONE = O_FULL + 1,
+  NUM_BARS = MIX_DONE + 1
 };
 
 struct __align__(64) Params {
   CUtensorMap p_maps[8];   // BSR values viewed [capacity * 64 lines][64]; box {64, 8 * (i + 1)}
-  CUtensorMap v_map;       // V viewed [n][H_r * d_v]; box {64, 64}
+  CUtensorMap v_map;       // V viewed [head-halves][n][64]; box {64, 64, d_v / 64}
   const int32_t* cu;
   SeqTables tab;
   const int32_t* row_ptr;
@@ -97,7 +130,7 @@ struct __align__(64) Params {
   const float* W;
   float* out;
   unsigned int* status;
-  int H_s, H_r, d_v, C, NR, KH, RB;
+  int H_s, H_r, d_v, C, NR, KH, RB, NP;
   uint32_t off_p, off_w, off_scr, off_recv, off_v, off_wf, off_bar;
 };
 
@@ -114,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int C = p.C;
+  const int NP = p.NP;
   const uint32_t crank = tc::cluster_rank();
   const int item = blockIdx.x / C;
   const int2 it = p.tab.items[item];
@@ -136,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
   if (tid == 0) {
     for (int i = 0; i < NUM_BARS; ++i) {
       uint32_t cnt = 1;
-      if (i >= D_EMPTY && i < D_EMPTY + kND) cnt = 4;
+      if (i >= D_EMPTY && i < D_EMPTY + kNG) cnt = 4;
       if (i >= BUF_FREE && i < BUF_FREE + 2) cnt = (uint32_t)C;
       tc::mbar_init(bar_addr(bars, i), cnt);
     }
@@ -145,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
   }
   {
     uint4* z = reinterpret_cast<uint4*>(smem + p.off_p);
-    const int nz = (int)((kNP * p_stage + 1024u) / 16);
+    const int nz = (int)((NP * p_stage + 1024u) / 16);
     for (int i = tid; i < nz; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
     float* wf = reinterpret_cast<float*>(smem + p.off_wf);   // W transposed: [H_s][H_r]
     for (int i = tid; i < p.H_r * p.H_s; i += kThreads) {
@@ -161,10 +195,12 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
   tc::cluster_sync();  // every CTA's barriers exist before any remote copy or arrival
   const uint32_t tmem = misc[0];
 
-  if (warp == 0) {
-    // ------------------------------ sender slices ------------------------------
+  if (warp == 0 || (warp >= 8 && warp < 8 + kPWarps - 1)) {
+    // ------------------------------ sender slices (chunks round-robin over 4 warps) ------------
+    const int pw = warp == 0 ? 0 : warp - 7;
+    const int nch = c1 - c0;
+    int q = 0, last = -1;
     if (lane == 0) {
-      int q = 0;
       unsigned long long m_next = T > 0 ? p.headmask[u0] : 0ull;
       int64_t off_next = T > 0 ? p.val_off[u0] : 0;
       for (int t = 0; t < T; ++t) {
@@ -177,16 +213,23 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         const int k = __popcll(m);
         const int k8 = (k + 7) >> 3;
         const int y0 = (int)(off * 64);   // first line of the block
-        for (int ch = c0; ch < c1; ++ch, ++q) {
-          const int ps = q % kNP;
-          if (q >= kNP) tc::wait_bar(bar_addr(bars, P_EMPTY + ps), ((q / kNP) - 1) & 1, abort_flag, p.status);
-          const uint32_t dst = sbase + p.off_p + ps * p_stage;
+        for (int c = 0; c < nch; ++c, ++q) {
+          if (q % kPWarps != pw) continue;
+          const int ps = q % NP;
+          if (q >= NP) tc::wait_bar(bar_addr(bars, P_EMPTY + ps), ((q / NP) - 1) & 1, abort_flag, p.status);
           tc::mbar_expect_tx(bar_addr(bars, P_FULL + ps), 2u * (uint32_t)k8 * 8u * 128u);
-          tc::tma_load_2d(dst, &p.p_maps[k8 - 1], 0, y0 + (2 * ch) * k, bar_addr(bars, P_FULL + ps));
-          tc::tma_load_2d(dst + p_box, &p.p_maps[k8 - 1], 0, y0 + (2 * ch + 1) * k,
+          const uint32_t dst = sbase + p.off_p + ps * p_stage;
+          tc::tma_load_2d(dst, &p.p_maps[k8 - 1], 0, y0 + (2 * (c0 + c)) * k, bar_addr(bars, P_FULL + ps));
+          tc::tma_load_2d(dst + p_box, &p.p_maps[k8 - 1], 0, y0 + (2 * (c0 + c) + 1) * k,
                           bar_addr(bars, P_FULL + ps));
+          last = q;
         }
       }
+      // drain: the final load of every slot, where this warp issued it, has landed (earlier uses
+      // of a slot are two phases back and must not be waited on)
+      for (int qq = max(0, q - NP); qq < q; ++qq)
+        if (qq % kPWarps == pw) tc::drain_bar(bar_addr(bars, P_FULL + qq % NP), (qq / NP) & 1);
+      (void)last;
     }
   } else if (warp == 7) {
     // ------------------------------ W' of each stored block ------------------------------
@@ -235,44 +278,80 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
       if (lane == 0) tc::mbar_arrive(bar_addr(bars, W_FULL + ws));
       __syncwarp();
     }
-  } else if (warp == 6) {
-    // ------------------------------ V tiles ------------------------------
+  } else if (warp == 6 || warp == 11) {
+    // ------------------------------ V tiles (receiver heads alternating over 2 warps) ----------
+    // slot rl holds V_rl[J] of the current block; it is refilled once this CTA's P.V of the
+    // previous block has completed (PV_DONE), so each slot is used once per block
+    const int vw = warp == 6 ? 0 : 1;
+    const int halves = p.d_v / 64;
     if (lane == 0) {
-      int vq = 0;
       int J_next = T > 0 ? p.col_idx[u0] : 0;
       for (int t = 0; t < T; ++t) {
         const int J = J_next;
         if (t + 1 < T) J_next = p.col_idx[u0 + t + 1];
-        for (int rl = 0; rl < G; ++rl, ++vq) {
-          const int vs = vq % kNV;
-          if (vq >= kNV) tc::wait_bar(bar_addr(bars, V_EMPTY + vs), ((vq / kNV) - 1) & 1, abort_flag, p.status);
-          const uint32_t dst = sbase + p.off_v + vs * v_stage;
-          tc::mbar_expect_tx(bar_addr(bars, V_FULL + vs), v_stage);
-          const int x = (r0 + rl) * p.d_v, y = seq0 + J * 64;
-          tc::tma_load_2d(dst, &p.v_map, x, y, bar_addr(bars, V_FULL + vs));
-          if (p.d_v == 128) tc::tma_load_2d(dst + 8192u, &p.v_map, x + 64, y, bar_addr(bars, V_FULL + vs));
+        if (t >= 1) tc::wait_bar(bar_addr(bars, PV_DONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, abort_flag, p.status);
+        for (int rl = vw; rl < G; rl += kVWarps) {
+          tc::mbar_expect_tx(bar_addr(bars, V_FULL + rl), v_stage);
+          tc::tma_load_3d(sbase + p.off_v + rl * v_stage, &p.v_map, 0, seq0 + J * 64,
+                          (r0 + rl) * halves, bar_addr(bars, V_FULL + rl));
         }
       }
+      if (T > 0)
+        for (int rl = vw; rl < G; rl += kVWarps) tc::drain_bar(bar_addr(bars, V_FULL + rl), (T - 1) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------ MMA issue ------------------------------
+    // ------------------------------ mixing MMAs ------------------------------
     if (lane == 0) {
       const uint32_t id_mix = tc::idesc_bf16(128, p.NR, 1, 0);
+      const int nch = c1 - c0;
+      int q = 0, gq = 0;
+      int k_next = T > 0 ? __popcll(p.headmask[u0]) : 0;
+      for (int t = 0; t < T; ++t) {
+        const int ksteps = (k_next + 15) >> 4;
+        if (t + 1 < T) k_next = __popcll(p.headmask[u0 + t + 1]);
+        const int ws = t & 1;
+        tc::wait_bar(bar_addr(bars, W_FULL + ws), (t >> 1) & 1, abort_flag, p.status);
+        const uint32_t wb = sbase + p.off_w + ws * w_stage;
+        for (int c = 0; c < nch; c += 2, ++gq) {
+          const int gs = gq % kNG;
+          if (gq >= kNG) tc::wait_bar(bar_addr(bars, D_EMPTY + gs), ((gq / kNG) - 1) & 1, abort_flag, p.status);
+          const int nj = min(2, nch - c);
+          for (int j = 0; j < nj; ++j) {
+            const int qq = q + c + j, ps = qq % NP;
+            tc::wait_bar(bar_addr(bars, P_FULL + ps), (qq / NP) & 1, abort_flag, p.status);
+            tc::tc_fence_after();
+            const uint32_t pa = sbase + p.off_p + ps * p_stage;
+            const uint32_t d = tmem + (uint32_t)kMixCol + (uint32_t)(2 * gs + j) * (uint32_t)p.NR;
+            for (int kk = 0; kk < ksteps; ++kk) {
+              const uint64_t a = tc::sdesc_sw128(pa + kk * 2048u, p_box, 1024u);
+              const uint64_t b = tc::sdesc_sw128(wb + kk * 32u, 16u, 1024u);
+              tc::mma_bf16(d, a, b, id_mix, kk > 0 ? 1u : 0u);
+            }
+          }
+          tc::mma_commit(bar_addr(bars, D_FULL + gs));
+        }
+        q += nch;
+        tc::mma_commit(bar_addr(bars, W_EMPTY + ws));
+      }
+      tc::mma_commit(bar_addr(bars, MIX_DONE));
+      tc::drain_bar(bar_addr(bars, MIX_DONE), 0);   // every mixing MMA completed before TMEM is freed
+    }
+  } else if (warp == 12) {
+    // ------------------------------ P.V MMAs ------------------------------
+    if (lane == 0) {
       const uint32_t id_pv = tc::idesc_bf16(128, 64, 1, 0);
       const uint32_t v_lbo = p.d_v == 128 ? 8192u : 0u;
       const uint16_t all_ctas = (uint16_t)((1u << C) - 1u);
-      int q = 0, vq = 0;
-      auto pv = [&](int t) {
+      for (int t = 0; t < T; ++t) {
         const int rs = t & 1;
         tc::mbar_expect_tx(bar_addr(bars, RECV_FULL + rs), (uint32_t)G * 8192u);
         tc::wait_bar(bar_addr(bars, RECV_FULL + rs), (t >> 1) & 1, abort_flag, p.status);
         tc::tc_fence_after();
         tc::fence_proxy_async_smem();  // peers' st.async data, read next by the tensor cores
-        for (int rl = 0; rl < G; ++rl, ++vq) {
-          const int vs = vq % kNV;
-          tc::wait_bar(bar_addr(bars, V_FULL + vs), (vq / kNV) & 1, abort_flag, p.status);
+        for (int rl = 0; rl < G; ++rl) {
+          tc::wait_bar(bar_addr(bars, V_FULL + rl), t & 1, abort_flag, p.status);
           tc::tc_fence_after();
-          const uint32_t va = sbase + p.off_v + vs * v_stage;
+          const uint32_t va = sbase + p.off_v + rl * v_stage;
           const uint32_t pb = sbase + p.off_recv + (uint32_t)rs * (kG * 8192u) + (uint32_t)rl * 8192u;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
@@ -280,38 +359,12 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
             const uint64_t b = tc::sdesc_sw128(pb + kk * 32u, 16u, 1024u);
             tc::mma_bf16(tmem + (uint32_t)rl * 64u, a, b, id_pv, (t > 0 || kk > 0) ? 1u : 0u);
           }
-          tc::mma_commit(bar_addr(bars, V_EMPTY + vs));
         }
+        tc::mma_commit(bar_addr(bars, PV_DONE + rs));
         tc::mma_commit_to_cluster(bar_addr(bars, BUF_FREE + rs), all_ctas);
-      };
-      int k_next = T > 0 ? __popcll(p.headmask[u0]) : 0;
-      for (int t = 0; t < T; ++t) {
-        const int ksteps = (k_next + 15) >> 4;
-        if (t + 1 < T) k_next = __popcll(p.headmask[u0 + t + 1]);
-        const int ws = t & 1;
-        tc::wait_bar(bar_addr(bars, W_FULL + ws), (t >> 1) & 1, abort_flag, p.status);
-        tc::tc_fence_after();
-        const uint32_t wb = sbase + p.off_w + ws * w_stage;
-        for (int ch = c0; ch < c1; ++ch, ++q) {
-          const int ps = q % kNP, ds = q % kND;
-          tc::wait_bar(bar_addr(bars, P_FULL + ps), (q / kNP) & 1, abort_flag, p.status);
-          if (q >= kND) tc::wait_bar(bar_addr(bars, D_EMPTY + ds), ((q / kND) - 1) & 1, abort_flag, p.status);
-          tc::tc_fence_after();
-          const uint32_t pa = sbase + p.off_p + ps * p_stage;
-          const uint32_t d = tmem + (uint32_t)kMixCol + (uint32_t)ds * (uint32_t)p.NR;
-          for (int kk = 0; kk < ksteps; ++kk) {
-            const uint64_t a = tc::sdesc_sw128(pa + kk * 2048u, p_box, 1024u);
-            const uint64_t b = tc::sdesc_sw128(wb + kk * 32u, 16u, 1024u);
-            tc::mma_bf16(d, a, b, id_mix, kk > 0 ? 1u : 0u);
-          }
-          tc::mma_commit(bar_addr(bars, P_EMPTY + ps));
-          tc::mma_commit(bar_addr(bars, D_FULL + ds));
-        }
-        tc::mma_commit(bar_addr(bars, W_EMPTY + ws));
-        if (t > 0) pv(t - 1);
       }
-      if (T > 0) pv(T - 1);
       tc::mma_commit(bar_addr(bars, O_FULL));
+      tc::drain_bar(bar_addr(bars, O_FULL), 0);   // every P.V MMA completed before TMEM is freed
     }
   } else {
     // ------------------------------ readout, exchange, output (warps 2-5) ------------------------------
@@ -320,19 +373,26 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
     unsigned char* scr = smem + p.off_scr + (warp - 2) * 2048;   // [32 heads][32 positions] bf16
     const int o = lane & 3;               // this lane's 16-byte run: positions 8*o .. 8*o+7
     const int rq = lane >> 2;             // this lane's heads: 8*v + rq
-    int q = 0;
+    const int nch = c1 - c0;
+    int q = 0, gq = 0;
     for (int t = 0; t < T; ++t) {
       const int ss = t & 1;
       // the receive buffers of round t-2 are free once every peer's P.V of that round completed
       if (t >= 2) tc::wait_bar(bar_addr(bars, BUF_FREE + ss), ((t - 2) >> 1) & 1, abort_flag, p.status);
       const uint32_t recv_local = sbase + p.off_recv + (uint32_t)ss * (kG * 8192u);
       const uint32_t rbar_local = bar_addr(bars, RECV_FULL + ss);
-      for (int ch = c0; ch < c1; ++ch, ++q) {
-        const int ds = q % kND;
-        tc::wait_bar(bar_addr(bars, D_FULL + ds), (q / kND) & 1, abort_flag, p.status);
+      for (int cc = 0; cc < nch; ++cc) {
+        const int gs = gq % kNG, j = cc & 1;
+        const int ch = c0 + cc;
+        if (j == 0) {
+          tc::wait_bar(bar_addr(bars, D_FULL + gs), (gq / kNG) & 1, abort_flag, p.status);
+          // the pair's mixing MMAs completed: their sender slots can be refilled
+          if (warp == 2 && lane == 0)
+            for (int jj = 0; jj < min(2, nch - cc); ++jj) tc::mbar_arrive(bar_addr(bars, P_EMPTY + (q + cc + jj) % NP));
+        }
         tc::tc_fence_after();
         uint32_t v[32];
-        const uint32_t ta = tmem + lane_base + (uint32_t)kMixCol + (uint32_t)ds * (uint32_t)p.NR;
+        const uint32_t ta = tmem + lane_base + (uint32_t)kMixCol + (uint32_t)(2 * gs + j) * (uint32_t)p.NR;
         if (p.NR == 32) {
           IAMAP_TMEM_LD32(ta, v);
         } else {
@@ -341,9 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
           for (int i = 16; i < 32; ++i) v[i] = 0u;
         }
         tc::tmem_ld_wait();
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(bar_addr(bars, D_EMPTY + ds));
+        if (j == 1 || cc + 1 == nch) {
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(bar_addr(bars, D_EMPTY + gs));
+          ++gq;
+        }
         // transpose: position = lane, head = register  ->  16-byte runs of one head
 #pragma unroll
         for (int r = 0; r < 32; ++r)
@@ -366,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         }
         __syncwarp();
       }
+      q += nch;
     }
     // output rows: TMEM lane = d_v index, column = rl * 64 + row of the block
     tc::wait_bar(bar_addr(bars, O_FULL), 0, abort_flag, p.status);
@@ -419,9 +483,16 @@ int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream) {
   p.NR = a.H_r <= 16 ? 16 : 32;
   p.KH = (a.H_s + 15) / 16 * 16;
   p.RB = (a.H_s + 7) / 8 * 8;
+  // everything but the sender ring, then as many ring slots as fit (at most kMaxNP)
+  const size_t fixed = (size_t)2 * p.NR * 128 + 1024 + (size_t)2 * kG * 8192 + (size_t)kNV * a.d_v * 128 +
+                       (size_t)4 * 2048 + sizeof(float) * (size_t)a.H_r * a.H_s + 8 * NUM_BARS + 96 + 4096;
+  const size_t p_stage_b = (size_t)2 * p.RB * 128;
+  const size_t budget = 232448 - 1024;
+  p.NP = (int)std::min<size_t>(kMaxNP, (budget - fixed - 1024) / p_stage_b);
+  if (p.NP < 2) return set_error(IAMAP_ERR_UNSUPPORTED, "mapped_av: sender ring does not fit");
   size_t off = 0;
   p.off_p = (uint32_t)off;
-  off += (size_t)kNP * 2 * p.RB * 128 + 1024;   // ring + tail read past the last box
+  off += (size_t)p.NP * p_stage_b + 1024;   // ring + tail read past the last box
   off = round_up(off, 1024);
   p.off_w = (uint32_t)off;
   off += (size_t)2 * p.NR * 128;
@@ -446,8 +517,8 @@ int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream) {
     int rc = encode_tmap_2d_bf16(&p.p_maps[i], a.vals, 64, cap * 64, 128, 64, (uint32_t)(8 * (i + 1)));
     if (rc) return rc;
   }
-  int rc = encode_tmap_2d_bf16(&p.v_map, a.v, (uint64_t)a.H_r * a.d_v, (uint64_t)a.n,
-                               (uint64_t)a.H_r * a.d_v * 2, 64, 64);
+  int rc = encode_tmap_3d_bf16(&p.v_map, a.v, 64, (uint64_t)a.n, (uint64_t)a.H_r * (a.d_v / 64),
+                               (uint64_t)a.H_r * a.d_v * 2, 128, 64, 64, (uint32_t)(a.d_v / 64));
   if (rc) return rc;
   p.cu = a.cu_seqlens;
   p.tab = a.tab;
