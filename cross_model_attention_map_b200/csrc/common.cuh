@@ -49,6 +49,8 @@ struct SeqTables {
   int32_t* cb_start;  // [num_seqs + 1]  (fits int32: checked on the host)
   int2* items;        // [num_rowblocks] (seq, I), longest causal row first
   int64_t* row_tiles; // [num_rowblocks] tiles of each row block (then their exclusive scan)
+  int2* pairs;        // [num_pairs] (seq, I0) of the row-block pairs (I0, I0 + 1), I0 even,
+                      // longest first
 };
 size_t seq_tables_bytes(int num_seqs, int64_t num_rowblocks);
 SeqTables carve_seq_tables(void* ws, int num_seqs, int64_t num_rowblocks);
@@ -58,6 +60,7 @@ struct Plan {
   int64_t num_rowblocks = 0;
   int64_t num_causal_blocks = 0;
   int32_t max_nb = 0;
+  int64_t num_pairs = 0;   // sum over sequences of ceil(nb / 2)
 };
 int make_plan(const int32_t* cu_host, int num_seqs, int B, int64_t n, Plan* out);
 

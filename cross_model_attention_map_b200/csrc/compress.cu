@@ -456,8 +456,9 @@ int compress_stats_impl(const CompressArgs& a, cudaStream_t stream) {
   IAMAP_CUDA_CHECK(cudaMemsetAsync(a.headmask_dense, 0,
                                    sizeof(uint64_t) * (size_t)a.plan.num_causal_blocks, stream));
   const size_t smem = stats_smem_bytes(a.d, a.plan.max_nb);
-  int rc = a.d == 64 ? launch_compress_kernel<64, false>(p, a.plan.num_rowblocks, smem, stream)
-                     : launch_compress_kernel<128, false>(p, a.plan.num_rowblocks, smem, stream);
+  int rc = compress_tc_supported(a.d, a.plan.max_nb) ? compress_stats_tc_launch(a, stream)
+           : a.d == 64 ? launch_compress_kernel<64, false>(p, a.plan.num_rowblocks, smem, stream)
+                       : launch_compress_kernel<128, false>(p, a.plan.num_rowblocks, smem, stream);
   if (rc) return rc;
   const int64_t nrb = a.plan.num_rowblocks;
   const unsigned wgrid = (unsigned)((nrb * 32 + 255) / 256);
@@ -494,8 +495,9 @@ int compress_extract_impl(const CompressArgs& a, cudaStream_t stream) {
   p.capacity = a.capacity;
   p.status = a.status;
   const size_t smem = extract_smem_bytes(a.d, a.plan.max_nb);
-  int rc = a.d == 64 ? launch_compress_kernel<64, true>(p, a.plan.num_rowblocks, smem, stream)
-                     : launch_compress_kernel<128, true>(p, a.plan.num_rowblocks, smem, stream);
+  int rc = compress_tc_supported(a.d, a.plan.max_nb) ? compress_extract_tc_launch(a, stream)
+           : a.d == 64 ? launch_compress_kernel<64, true>(p, a.plan.num_rowblocks, smem, stream)
+                       : launch_compress_kernel<128, true>(p, a.plan.num_rowblocks, smem, stream);
   if (rc) return rc;
   if (a.capacity > 0) {
     zero_tail_kernel<<<64, 256, 0, stream>>>(p.vals, a.counts_in, a.capacity);

@@ -1,0 +1,694 @@
+// map_compress on the 5th-generation tensor cores (tcgen05, TMEM accumulators, TMA operand loads).
+//
+// Same two stages as compress.cu (MapFlow news page, "PKU MapFlow: cross-model attention map
+// reuse", storage-and-execution part, first component: block statistics first, then extraction
+// of the blocks kept by cumulative attention probability), with the work of one CTA widened to a
+// pair of row blocks (I0 = 2P, I1 = 2P + 1: 128 query rows, one per TMEM lane) of one sender head.
+//
+// Stage 1 (stats_tc_kernel): S = Q K^T for 128 keys at a time (column blocks 2T, 2T + 1) lands in
+// one of two 128-column TMEM buffers. Eight softmax warps read it back, one thread per (row,
+// column block): the block's log2-sum c_iJ = log2 sum_j 2^(s_ij log2(e)/sqrt(d)) is kept in TMEM
+// column 256 + J, and the row's running log-sum-exp in registers. Afterwards the same threads
+// form lse_i, the block masses sum_i 2^(c_iJ - lse_i) (a 32 x 32 butterfly per warp sums over
+// rows), and the cumulative-mass choice of each row block. Rows with more than 256 column blocks
+// (sequences longer than 16384 tokens) take the mma.sync kernel instead.
+//
+// Stage 2 (extract_tc_kernel): for every column block J that this head keeps in I0 or I1,
+// S = Q K_J^T (128 x 64) is recomputed into TMEM; two groups of four warps take alternate blocks
+// and write exp(s - lse) as bf16 rows of the stored tiles, through a per-warp staging buffer so
+// that each 128-byte tile row leaves as one coalesced run (rows of the k present heads of a
+// stored block are interleaved: row i of head rank t is line i * k + t of the block).
+//
+// Roles (320 threads): warps 0-7 softmax / writers, warp 8 TMA producer, warp 9 MMA issuer (and
+// TMEM owner). Every wait is bounded (2 s; then IAMAP_DEV_TIMEOUT and an orderly exit).
+#include <algorithm>
+
+#include "tc_utils.cuh"
+#include "internal.h"
+
+namespace iamap {
+namespace tccomp {
+
+constexpr int kRows = 128;         // query rows per CTA (row blocks 2P, 2P + 1)
+constexpr int kThreads = 320;      // warps 0-7 softmax, 8 TMA, 9 MMA
+constexpr int kSoft = 256;         // softmax threads
+constexpr int kSStages = 4;        // stats: key-tile ring (128 keys per tile)
+constexpr int kXStages = 2;        // extract: key-tile ring (64 keys per tile)
+constexpr int kCCol = 256;         // stats: TMEM column of c_i0
+constexpr int kMaxNb = 256;        // stats: column blocks per row kept in TMEM
+constexpr uint32_t kPanel128 = 128u * 128u;   // 128 rows x 64 bf16 (one 128-byte swizzle span)
+constexpr uint32_t kPanel64 = 64u * 128u;
+
+enum { Q_FULL = 0, K_FULL = 1, K_EMPTY = K_FULL + kSStages, S_FULL = K_EMPTY + kSStages,
+       S_EMPTY = S_FULL + 2, NUM_BARS = S_EMPTY + 2 };
+constexpr int kXBufs = 4;          // extract: S buffers of 64 TMEM columns (two per writer group)
+enum { XQ_FULL = 0, XK_FULL = 1, XK_EMPTY = XK_FULL + kXStages, XS_FULL = XK_EMPTY + kXStages,
+       XS_EMPTY = XS_FULL + kXBufs, X_NUM_BARS = XS_EMPTY + kXBufs };
+
+struct StatsParams {
+  CUtensorMap q_map;   // {64, n, H_s * D / 64} bf16, box {64, 128, 1}
+  CUtensorMap k_map;   // same geometry
+  const int32_t* cu;
+  SeqTables tab;
+  int64_t n, ncb;
+  int H_s;
+  float scale_log2;
+  int bias_window;
+  float bias_log2;
+  float tau;
+  float* lse;
+  float* mass;
+  unsigned long long* headmask_dense;
+  unsigned int* status;
+};
+
+struct ExtractParams {
+  CUtensorMap q_map;   // box {64, 128, 1}
+  CUtensorMap k_map;   // box {64, 64, 1}
+  const int32_t* cu;
+  SeqTables tab;
+  int64_t n;
+  int H_s;
+  float scale_log2;
+  int bias_window;
+  float bias_log2;
+  const float* lse;
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  const unsigned long long* headmask;
+  const int64_t* val_off;
+  __nv_bfloat16* vals;
+  int64_t capacity;
+  unsigned int* status;
+};
+
+__device__ __forceinline__ uint32_t bar_addr(uint32_t bars, int i) { return bars + 8u * (uint32_t)i; }
+
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float x) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(x))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// x[e] = this lane's value of column e; returns the sum over the warp's 32 lanes of column
+// `lane` (31 shuffles: each step halves the columns a lane holds).
+__device__ __forceinline__ float transpose_sum32(float (&x)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int e = 0; e < w; ++e) {
+      const float send = upper ? x[e] : x[e + w];
+      const float keep = upper ? x[e + w] : x[e];
+      x[e] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return x[0];
+}
+
+// Exclusive prefix sums of x[0..n) (n <= 256) in place, by one warp.
+__device__ __forceinline__ void warp_exclusive_scan256(float* x, int n, int lane) {
+  float loc[8];
+  float tot = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int idx = lane * 8 + e;
+    const float v = idx < n ? x[idx] : 0.f;
+    loc[e] = tot;
+    tot += v;
+  }
+  float inc = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  const float base = inc - tot;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int idx = lane * 8 + e;
+    if (idx < n) x[idx] = base + loc[e];
+  }
+}
+
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
+  const uint32_t a = smem_u32(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Stage 1: block statistics, masses and the per-head choice
+// ------------------------------------------------------------------------------------------------
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_constant__ StatsParams p) {
+  constexpr int NPAN = D / 64;
+  constexpr uint32_t kQBytes = NPAN * kPanel128;
+  constexpr uint32_t kKStage = NPAN * kPanel128;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase, sK = sbase + kQBytes;
+  float* aux = reinterpret_cast<float*>(smem + kQBytes + kSStages * kKStage);
+  float* ml_m = aux;                  // [2][128] running max (log2) of each group
+  float* ml_l = ml_m + 2 * kRows;     // [2][128] running sum
+  float* lse_s = ml_l + 2 * kRows;    // [128] row lse (log2)
+  float* part = lse_s + kRows;        // [4][256] per-quarter column sums
+  float* mass_s = part + 4 * kMaxNb;  // [2][256]
+  float* sorted_s = mass_s + 2 * kMaxNb;
+  int* rank_s = reinterpret_cast<int*>(sorted_s + 2 * kMaxNb);
+  uint64_t* bar_mem = reinterpret_cast<uint64_t*>(rank_s + 2 * kMaxNb);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bar_mem + NUM_BARS);   // [0] tmem, [1] abort
+  const uint32_t bars = smem_u32(bar_mem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int pair = blockIdx.x / p.H_s;
+  const int h = blockIdx.x - pair * p.H_s;
+  const int2 it = p.tab.pairs[pair];
+  const int s = it.x, I0 = it.y, P = I0 >> 1;
+  const int seq0 = p.cu[s];
+  const int L = p.cu[s + 1] - seq0;
+  const int nb = p.tab.nb[s];
+  const int nT = P + 1;                     // key tiles of 128
+
+  if (tid == 0) {
+    for (int i = 0; i < NUM_BARS; ++i)
+      tc::mbar_init(bar_addr(bars, i), (i >= S_EMPTY && i < S_EMPTY + 2) ? 8u : 1u);
+    misc[1] = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 9) tc::tmem_alloc(smem_u32(misc), 512);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 8) {
+    // ------------------------------ TMA: Q once, then the key tiles ------------------------------
+    if (lane == 0) {
+      tc::mbar_expect_tx(bar_addr(bars, Q_FULL), kQBytes);
+#pragma unroll
+      for (int pan = 0; pan < NPAN; ++pan)
+        tc::tma_load_3d(sQ + pan * kPanel128, &p.q_map, 0, seq0 + kRows * P, h * NPAN + pan,
+                        bar_addr(bars, Q_FULL));
+      for (int T = 0; T < nT; ++T) {
+        const int st = T % kSStages;
+        if (T >= kSStages)
+          tc::wait_bar(bar_addr(bars, K_EMPTY + st), ((T / kSStages) - 1) & 1, abort_flag, p.status);
+        tc::mbar_expect_tx(bar_addr(bars, K_FULL + st), kKStage);
+#pragma unroll
+        for (int pan = 0; pan < NPAN; ++pan)
+          tc::tma_load_3d(sK + st * kKStage + pan * kPanel128, &p.k_map, 0, seq0 + 128 * T,
+                          h * NPAN + pan, bar_addr(bars, K_FULL + st));
+      }
+      for (int T = max(0, nT - kSStages); T < nT; ++T)
+        tc::drain_bar(bar_addr(bars, K_FULL + T % kSStages), (T / kSStages) & 1);
+      tc::drain_bar(bar_addr(bars, Q_FULL), 0);
+    }
+  } else if (warp == 9) {
+    // ------------------------------ MMA: S_b = Q K_T^T (128 x 128, fp32 in TMEM) ----------------
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 0);
+      tc::wait_bar(bar_addr(bars, Q_FULL), 0, abort_flag, p.status);
+      for (int T = 0; T < nT; ++T) {
+        const int st = T % kSStages, b = T & 1;
+        tc::wait_bar(bar_addr(bars, K_FULL + st), (T / kSStages) & 1, abort_flag, p.status);
+        if (T >= 2) tc::wait_bar(bar_addr(bars, S_EMPTY + b), ((T - 2) >> 1) & 1, abort_flag, p.status);
+        tc::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * kPanel128 + (uint32_t)(kk & 3) * 32u;
+          const uint64_t a = tc::sdesc_sw128(sQ + off, 16u, 1024u);
+          const uint64_t bd = tc::sdesc_sw128(sK + st * kKStage + off, 16u, 1024u);
+          tc::mma_bf16(tmem + (uint32_t)b * 128u, a, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(bar_addr(bars, K_EMPTY + st));
+        tc::mma_commit(bar_addr(bars, S_FULL + b));
+      }
+      if (nT > 0) tc::drain_bar(bar_addr(bars, S_FULL + ((nT - 1) & 1)), ((nT - 1) >> 1) & 1);
+    }
+  } else {
+    // ------------------------------ softmax: one thread per (row, column block) -----------------
+    const int qd = warp & 3, g = warp >> 2;
+    const int r = 32 * qd + lane;                 // TMEM lane = pair-local row
+    const int Ir = I0 + (r >> 6);                 // row block (uniform over the warp)
+    const int i = kRows * P + r;                  // sequence-local row
+    const bool valid = i < L;
+    const uint32_t t_lane = (uint32_t)(32 * qd) << 16;
+    const float sc = p.scale_log2;
+    float m_acc = -INFINITY, l_acc = 0.f;
+    for (int T = 0; T < nT; ++T) {
+      const int b = T & 1;
+      const int J = 2 * T + g;
+      tc::wait_bar(bar_addr(bars, S_FULL + b), (T >> 1) & 1, abort_flag, p.status);
+      tc::tc_fence_after();
+      uint32_t v[64];
+      if (J <= Ir) {
+        IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(b * 128 + g * 64), v);
+        IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(b * 128 + g * 64 + 32), (v + 32));
+        tc::tmem_ld_wait();
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_addr(bars, S_EMPTY + b));
+      if (J > Ir) continue;
+      const int j0 = 64 * J;
+      float c;
+      if (J < Ir && !(p.bias_window > 0 && i - j0 - 63 < p.bias_window)) {
+        // no causal mask and no bias inside this block
+        float mx = __uint_as_float(v[0]);
+#pragma unroll
+        for (int e = 1; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+        const float nm = -mx * sc;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+        for (int e = 0; e < 64; e += 4) {
+          s0 += ex2(fmaf(__uint_as_float(v[e]), sc, nm));
+          s1 += ex2(fmaf(__uint_as_float(v[e + 1]), sc, nm));
+          s2 += ex2(fmaf(__uint_as_float(v[e + 2]), sc, nm));
+          s3 += ex2(fmaf(__uint_as_float(v[e + 3]), sc, nm));
+        }
+        c = mx * sc + lg2((s0 + s1) + (s2 + s3));
+      } else {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          const int j = j0 + e;
+          float x = __uint_as_float(v[e]) * sc;
+          if (p.bias_window > 0 && i - j >= 0 && i - j < p.bias_window) x += p.bias_log2;
+          x = j > i ? -INFINITY : x;
+          v[e] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+        if (mx == -INFINITY) {
+          c = -INFINITY;
+        } else {
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            s0 += ex2(__uint_as_float(v[e]) - mx);
+            s1 += ex2(__uint_as_float(v[e + 1]) - mx);
+          }
+          c = mx + lg2(s0 + s1);
+        }
+      }
+      if (c > m_acc) {
+        l_acc = l_acc * ex2(m_acc - c) + 1.f;
+        m_acc = c;
+      } else if (c > -INFINITY) {
+        l_acc += ex2(c - m_acc);
+      }
+      tmem_st1(tmem + t_lane + (uint32_t)(kCCol + J), c);
+    }
+    tmem_st_wait();
+
+    // ---- row log-sum-exp (both groups' partial sums) ----
+    ml_m[g * kRows + r] = m_acc;
+    ml_l[g * kRows + r] = l_acc;
+    tc::tc_fence_before();
+    tc::named_bar(1, kSoft);
+    tc::tc_fence_after();
+    if (g == 0) {
+      const float m0 = ml_m[r], m1 = ml_m[kRows + r];
+      const float m = fmaxf(m0, m1);
+      float lse2 = -INFINITY;
+      if (m > -INFINITY) lse2 = m + lg2(ml_l[r] * ex2(m0 - m) + ml_l[kRows + r] * ex2(m1 - m));
+      lse_s[r] = lse2;
+      if (valid) p.lse[(int64_t)h * p.n + seq0 + i] = lse2 * kLn2;
+    }
+    tc::named_bar(1, kSoft);
+
+    // ---- block masses: sum over the valid rows of 2^(c_iJ - lse_i) ----
+    const int nJ = min(2 * P + 2, nb);
+    const float lr = lse_s[r];
+    for (int ch = g; ch * 32 < nJ; ch += 2) {
+      uint32_t cv[32];
+      IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(kCCol + 32 * ch), cv);
+      tc::tmem_ld_wait();
+      float x[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int J = 32 * ch + e;
+        x[e] = (valid && J <= Ir) ? ex2(__uint_as_float(cv[e]) - lr) : 0.f;
+      }
+      part[qd * kMaxNb + 32 * ch + lane] = transpose_sum32(x, lane);
+    }
+    tc::named_bar(1, kSoft);
+    for (int idx = tid; idx < 2 * kMaxNb; idx += kSoft) {
+      const int k = idx / kMaxNb, J = idx - k * kMaxNb;
+      const int I = I0 + k;
+      if (I < nb && J <= I) {
+        const float m = part[(2 * k) * kMaxNb + J] + part[(2 * k + 1) * kMaxNb + J];
+        mass_s[k * kMaxNb + J] = m;
+        p.mass[(int64_t)h * p.ncb + p.tab.cb_start[s] + (int64_t)I * (I + 1) / 2 + J] = m;
+      }
+    }
+    tc::named_bar(1, kSoft);
+
+    // ---- cumulative-mass choice per row block: decreasing mass (ties: lower J first); a block
+    // is kept while the mass before it is below tau * R ----
+    const unsigned long long bit = 1ull << h;
+    if (p.tau >= 1.f) {
+      for (int idx = tid; idx < 2 * kMaxNb; idx += kSoft) {
+        const int k = idx / kMaxNb, J = idx - k * kMaxNb, I = I0 + k;
+        if (I < nb && J <= I)
+          atomicOr(p.headmask_dense + p.tab.cb_start[s] + (int64_t)I * (I + 1) / 2 + J, bit);
+      }
+    } else {
+      for (int idx = tid; idx < 2 * kMaxNb; idx += kSoft) {
+        const int k = idx / kMaxNb, J = idx - k * kMaxNb, I = I0 + k;
+        if (I < nb && J <= I) {
+          const float* ms = mass_s + k * kMaxNb;
+          const float mJ = ms[J];
+          int rank = 0;
+          for (int J2 = 0; J2 <= I; ++J2) {
+            const float m2 = ms[J2];
+            rank += (m2 > mJ) || (m2 == mJ && J2 < J);
+          }
+          rank_s[k * kMaxNb + J] = rank;
+          sorted_s[k * kMaxNb + rank] = mJ;
+        }
+      }
+      tc::named_bar(1, kSoft);
+      if (warp < 2 && I0 + warp < nb) warp_exclusive_scan256(sorted_s + warp * kMaxNb, I0 + warp + 1, lane);
+      tc::named_bar(1, kSoft);
+      for (int idx = tid; idx < 2 * kMaxNb; idx += kSoft) {
+        const int k = idx / kMaxNb, J = idx - k * kMaxNb, I = I0 + k;
+        if (I < nb && J <= I) {
+          const float R = (float)min(64, L - 64 * I);
+          if (sorted_s[k * kMaxNb + rank_s[k * kMaxNb + J]] < p.tau * R)
+            atomicOr(p.headmask_dense + p.tab.cb_start[s] + (int64_t)I * (I + 1) / 2 + J, bit);
+        }
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Stage 2: extraction of the kept tiles
+// ------------------------------------------------------------------------------------------------
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_constant__ ExtractParams p) {
+  constexpr int NPAN = D / 64;
+  constexpr uint32_t kQBytes = NPAN * kPanel128;
+  constexpr uint32_t kKStage = NPAN * kPanel64;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase, sK = sbase + kQBytes;
+  unsigned char* stage_all = smem + kQBytes + kXStages * kKStage;        // 8 warps x 4 KB
+  int64_t* base_s = reinterpret_cast<int64_t*>(stage_all + 8 * 4096);    // [2][256] tile index
+  int* rk_s = reinterpret_cast<int*>(base_s + 2 * kMaxNb);               // [2][256] rank | k << 8
+  int* ulist = rk_s + 2 * kMaxNb;                                        // [256] union of J
+  uint64_t* bar_mem = reinterpret_cast<uint64_t*>(ulist + kMaxNb);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bar_mem + X_NUM_BARS);    // [0] tmem [1] abort [2] count
+  const uint32_t bars = smem_u32(bar_mem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int pair = blockIdx.x / p.H_s;
+  const int h = blockIdx.x - pair * p.H_s;
+  const int2 it = p.tab.pairs[pair];
+  const int s = it.x, I0 = it.y, P = I0 >> 1;
+  const int seq0 = p.cu[s];
+  const int L = p.cu[s + 1] - seq0;
+  const int nb = p.tab.nb[s];
+  const int nJ = min(2 * P + 2, nb);
+
+  if (tid == 0) {
+    for (int i = 0; i < X_NUM_BARS; ++i)
+      tc::mbar_init(bar_addr(bars, i), (i >= XS_EMPTY && i < XS_EMPTY + kXBufs) ? 4u : 1u);
+    misc[1] = 0;
+    tc::fence_barrier_init();
+  }
+  for (int idx = tid; idx < 2 * kMaxNb; idx += kThreads) base_s[idx] = -1;
+  if (warp == 9) tc::tmem_alloc(smem_u32(misc), 256);
+  __syncthreads();
+  // this head's stored blocks in row blocks I0 and I1, by column block
+  if (warp < 2 && I0 + warp < nb) {
+    const int rb = p.tab.rb_start[s] + I0 + warp;
+    const int u0 = p.row_ptr[rb], u1 = p.row_ptr[rb + 1];
+    const unsigned long long below = (1ull << h) - 1ull;
+    for (int u = u0 + lane; u < u1; u += 32) {
+      const unsigned long long m = p.headmask[u];
+      if ((m >> h) & 1ull) {
+        const int J = p.col_idx[u];
+        base_s[warp * kMaxNb + J] = p.val_off[u];
+        rk_s[warp * kMaxNb + J] = __popcll(m & below) | (__popcll(m) << 8);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int cnt = 0;
+    for (int J0 = 0; J0 < nJ; J0 += 32) {
+      const int J = J0 + lane;
+      const bool any = J < nJ && (base_s[J] >= 0 || base_s[kMaxNb + J] >= 0);
+      const unsigned bal = __ballot_sync(0xffffffffu, any);
+      if (any) ulist[cnt + __popc(bal & ((1u << lane) - 1u))] = J;
+      cnt += __popc(bal);
+    }
+    if (lane == 0) misc[2] = (uint32_t)cnt;
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int nU = (int)misc[2];
+
+  if (warp == 8) {
+    if (lane == 0) {
+      tc::mbar_expect_tx(bar_addr(bars, XQ_FULL), kQBytes);
+#pragma unroll
+      for (int pan = 0; pan < NPAN; ++pan)
+        tc::tma_load_3d(sQ + pan * kPanel128, &p.q_map, 0, seq0 + kRows * P, h * NPAN + pan,
+                        bar_addr(bars, XQ_FULL));
+      for (int t = 0; t < nU; ++t) {
+        const int st = t % kXStages;
+        if (t >= kXStages)
+          tc::wait_bar(bar_addr(bars, XK_EMPTY + st), ((t / kXStages) - 1) & 1, abort_flag, p.status);
+        tc::mbar_expect_tx(bar_addr(bars, XK_FULL + st), kKStage);
+        const int J = ulist[t];
+#pragma unroll
+        for (int pan = 0; pan < NPAN; ++pan)
+          tc::tma_load_3d(sK + st * kKStage + pan * kPanel64, &p.k_map, 0, seq0 + 64 * J,
+                          h * NPAN + pan, bar_addr(bars, XK_FULL + st));
+      }
+      for (int t = max(0, nU - kXStages); t < nU; ++t)
+        tc::drain_bar(bar_addr(bars, XK_FULL + t % kXStages), (t / kXStages) & 1);
+      tc::drain_bar(bar_addr(bars, XQ_FULL), 0);
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(128, 64, 0, 0);
+      tc::wait_bar(bar_addr(bars, XQ_FULL), 0, abort_flag, p.status);
+      for (int t = 0; t < nU; ++t) {
+        const int st = t % kXStages, b = t & (kXBufs - 1);
+        tc::wait_bar(bar_addr(bars, XK_FULL + st), (t / kXStages) & 1, abort_flag, p.status);
+        if (t >= kXBufs) tc::wait_bar(bar_addr(bars, XS_EMPTY + b), ((t - kXBufs) >> 2) & 1, abort_flag, p.status);
+        tc::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (uint32_t)(kk & 3) * 32u;
+          const uint64_t a = tc::sdesc_sw128(sQ + (uint32_t)(kk >> 2) * kPanel128 + ko, 16u, 1024u);
+          const uint64_t bd = tc::sdesc_sw128(sK + st * kKStage + (uint32_t)(kk >> 2) * kPanel64 + ko, 16u, 1024u);
+          tc::mma_bf16(tmem + (uint32_t)b * 64u, a, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(bar_addr(bars, XK_EMPTY + st));
+        tc::mma_commit(bar_addr(bars, XS_FULL + b));
+      }
+      if (nU > 0) tc::drain_bar(bar_addr(bars, XS_FULL + ((nU - 1) & (kXBufs - 1))), ((nU - 1) >> 2) & 1);
+    }
+  } else {
+    // ------------------------------ writers: group G takes the blocks t = G, G + 2, ... --------
+    const int qd = warp & 3, G = warp >> 2;
+    const int r = 32 * qd + lane;
+    const int kb = r >> 6;                        // 0: row block I0, 1: I1 (uniform over the warp)
+    const int Ir = I0 + kb;
+    const int i = kRows * P + r;
+    const bool valid = i < L;
+    const int il = r & 63;                        // row within the tile
+    const uint32_t t_lane = (uint32_t)(32 * qd) << 16;
+    const float sc = p.scale_log2;
+    const float lse2 = valid ? p.lse[(int64_t)h * p.n + seq0 + i] * kLog2e : 0.f;
+    unsigned char* stg = stage_all + warp * 4096;
+    bool cap_flag = false;
+    for (int t = G; t < nU; t += 2) {
+      const int b = t & (kXBufs - 1);
+      tc::wait_bar(bar_addr(bars, XS_FULL + b), (t >> 2) & 1, abort_flag, p.status);
+      tc::tc_fence_after();
+      const int J = ulist[t];
+      const int64_t base = base_s[kb * kMaxNb + J];
+      const int rk = rk_s[kb * kMaxNb + J];
+      const int rank = rk & 255, k = rk >> 8;
+      if (base >= 0) {
+        // exp(s - lse) of this row, 32 columns at a time, staged as bf16 (16-byte chunk c of
+        // the row at c ^ (row & 7))
+        const int j0 = 64 * J;
+        const bool fast = J < Ir && !(p.bias_window > 0 && i - j0 - 63 < p.bias_window);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
+          IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(b * 64 + 32 * half), v);
+          tc::tmem_ld_wait();
+          uint32_t pk[16];
+          if (fast) {
+            const float nl = -lse2;
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float a0 = valid ? ex2(fmaf(__uint_as_float(v[e]), sc, nl)) : 0.f;
+              const float a1 = valid ? ex2(fmaf(__uint_as_float(v[e + 1]), sc, nl)) : 0.f;
+              pk[e >> 1] = pack_bf16(a0, a1);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float a[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int j = j0 + 32 * half + e + u;
+                float x = __uint_as_float(v[e + u]) * sc;
+                if (p.bias_window > 0 && i - j >= 0 && i - j < p.bias_window) x += p.bias_log2;
+                a[u] = (valid && j <= i) ? ex2(x - lse2) : 0.f;
+              }
+              pk[e >> 1] = pack_bf16(a[0], a[1]);
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int cc = 4 * half + c;
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((cc ^ (lane & 7)) << 4)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_addr(bars, XS_EMPTY + b));
+      if (base < 0) continue;
+      // write 4 tile rows of 128 B per step
+      __syncwarp();
+      if (base + k <= p.capacity) {
+        __nv_bfloat16* blk = p.vals + base * (64 * 64) + (int64_t)rank * 64;
+        const int c = lane & 7;
+#pragma unroll
+        for (int step = 0; step < 8; ++step) {
+          const int row = 4 * step + (lane >> 3);          // warp-local row
+          const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 128 + ((c ^ (row & 7)) << 4));
+          const int tr = (il - lane) + row;                 // tile row of that warp-local row
+          *reinterpret_cast<uint4*>(blk + (int64_t)tr * k * 64 + c * 8) = val;
+        }
+      } else {
+        cap_flag = true;
+      }
+      __syncwarp();
+    }
+    if (cap_flag && lane == 0) raise_status(p.status, IAMAP_DEV_CAPACITY);
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int D>
+static size_t stats_smem() {
+  return 1024 + (size_t)(D / 64) * kPanel128 * (1 + kSStages) +
+         sizeof(float) * (2 * kRows + 2 * kRows + kRows + 4 * kMaxNb + 2 * kMaxNb + 2 * kMaxNb) +
+         sizeof(int) * 2 * kMaxNb + 8 * NUM_BARS + 16;
+}
+template <int D>
+static size_t extract_smem() {
+  return 1024 + (size_t)(D / 64) * (kPanel128 + kXStages * kPanel64) + 8 * 4096 +
+         sizeof(int64_t) * 2 * kMaxNb + sizeof(int) * 3 * kMaxNb + 8 * X_NUM_BARS + 16;
+}
+
+}  // namespace tccomp
+
+bool compress_tc_supported(int d, int max_nb) {
+  return (d == 64 || d == 128) && max_nb <= tccomp::kMaxNb;
+}
+
+static int encode_qk_map(CUtensorMap* map, const void* base, int64_t n, int H_s, int d, int box_rows) {
+  return encode_tmap_3d_bf16(map, base, 64, (uint64_t)n, (uint64_t)H_s * (d / 64),
+                             (uint64_t)H_s * d * 2, 128, 64, (uint32_t)box_rows, 1);
+}
+
+int compress_stats_tc_launch(const CompressArgs& a, cudaStream_t stream) {
+  using namespace tccomp;
+  StatsParams p{};
+  int rc = encode_qk_map(&p.q_map, a.q, a.n, a.H_s, a.d, 128);
+  if (!rc) rc = encode_qk_map(&p.k_map, a.k, a.n, a.H_s, a.d, 128);
+  if (rc) return rc;
+  p.cu = a.cu_seqlens;
+  p.tab = a.tab;
+  p.n = a.n;
+  p.ncb = a.plan.num_causal_blocks;
+  p.H_s = a.H_s;
+  p.scale_log2 = kLog2e / sqrtf((float)a.d);
+  p.bias_window = a.bias_window;
+  p.bias_log2 = a.bias_value * kLog2e;
+  p.tau = a.tau;
+  p.lse = a.lse;
+  p.mass = a.mass;
+  p.headmask_dense = reinterpret_cast<unsigned long long*>(a.headmask_dense);
+  p.status = a.status;
+  // one CTA per SM: it holds all 512 TMEM columns
+  const size_t smem = std::max<size_t>(a.d == 64 ? stats_smem<64>() : stats_smem<128>(), 120 * 1024);
+  auto kern = a.d == 64 ? stats_tc_kernel<64> : stats_tc_kernel<128>;
+  IAMAP_CUDA_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int64_t grid = a.plan.num_pairs * a.H_s;
+  if (grid > 0) {
+    kern<<<(unsigned)grid, kThreads, smem, stream>>>(p);
+    IAMAP_LAUNCH_CHECK("compress stats (tcgen05)");
+  }
+  return IAMAP_OK;
+}
+
+int compress_extract_tc_launch(const CompressArgs& a, cudaStream_t stream) {
+  using namespace tccomp;
+  ExtractParams p{};
+  int rc = encode_qk_map(&p.q_map, a.q, a.n, a.H_s, a.d, 128);
+  if (!rc) rc = encode_qk_map(&p.k_map, a.k, a.n, a.H_s, a.d, 64);
+  if (rc) return rc;
+  p.cu = a.cu_seqlens;
+  p.tab = a.tab;
+  p.n = a.n;
+  p.H_s = a.H_s;
+  p.scale_log2 = kLog2e / sqrtf((float)a.d);
+  p.bias_window = a.bias_window;
+  p.bias_log2 = a.bias_value * kLog2e;
+  p.lse = a.lse_in;
+  p.row_ptr = a.row_ptr_in;
+  p.col_idx = a.col_idx_in;
+  p.headmask = reinterpret_cast<const unsigned long long*>(a.headmask_in);
+  p.val_off = a.val_off_in;
+  p.vals = static_cast<__nv_bfloat16*>(a.vals);
+  p.capacity = a.capacity;
+  p.status = a.status;
+  const size_t smem = a.d == 64 ? extract_smem<64>() : extract_smem<128>();
+  auto kern = a.d == 64 ? extract_tc_kernel<64> : extract_tc_kernel<128>;
+  IAMAP_CUDA_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int64_t grid = a.plan.num_pairs * a.H_s;
+  if (grid > 0) {
+    kern<<<(unsigned)grid, kThreads, smem, stream>>>(p);
+    IAMAP_LAUNCH_CHECK("compress extract (tcgen05)");
+  }
+  return IAMAP_OK;
+}
+
+}  // namespace iamap

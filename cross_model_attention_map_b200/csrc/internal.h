@@ -41,6 +41,11 @@ struct CompressArgs {
 int compress_stats_impl(const CompressArgs& a, cudaStream_t stream);
 int compress_extract_impl(const CompressArgs& a, cudaStream_t stream);
 size_t compress_stats_smem(int d, int max_nb);
+// Tensor-core forms (compress_tc.cu), used when supported: d of 64 or 128, at most 256 column
+// blocks per sequence.
+bool compress_tc_supported(int d, int max_nb);
+int compress_stats_tc_launch(const CompressArgs& a, cudaStream_t stream);
+int compress_extract_tc_launch(const CompressArgs& a, cudaStream_t stream);
 size_t compress_extract_smem(int d, int max_nb);
 
 struct MappedAvArgs {

@@ -68,6 +68,7 @@ int make_plan(const int32_t* cu_host, int num_seqs, int B, int64_t n, Plan* out)
     int64_t nb = (L + B - 1) / B;
     p.num_rowblocks += nb;
     p.num_causal_blocks += nb * (nb + 1) / 2;
+    p.num_pairs += (nb + 1) / 2;
     if (nb > p.max_nb) p.max_nb = (int32_t)nb;
   }
   if (n >= 0 && (int64_t)cu_host[num_seqs] != n)
@@ -85,7 +86,8 @@ size_t seq_tables_bytes(int num_seqs, int64_t num_rowblocks) {
   return align256(sizeof(int32_t) * (size_t)num_seqs) +
          2 * align256(sizeof(int32_t) * (size_t)(num_seqs + 1)) +
          align256(sizeof(int2) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1)) +
-         align256(sizeof(int64_t) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1));
+         align256(sizeof(int64_t) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1)) +
+         align256(sizeof(int2) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1));
 }
 
 SeqTables carve_seq_tables(void* ws, int num_seqs, int64_t num_rowblocks) {
@@ -100,6 +102,8 @@ SeqTables carve_seq_tables(void* ws, int num_seqs, int64_t num_rowblocks) {
   t.items = reinterpret_cast<int2*>(p);
   p += align256(sizeof(int2) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1));
   t.row_tiles = reinterpret_cast<int64_t*>(p);
+  p += align256(sizeof(int64_t) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1));
+  t.pairs = reinterpret_cast<int2*>(p);   // at most num_rowblocks pairs
   return t;
 }
 
@@ -131,6 +135,18 @@ __global__ void build_tables_kernel(const int32_t* __restrict__ cu, int num_seqs
     int32_t c = 0;
     for (int s = 0; s < num_seqs; ++s)
       if (t.nb[s] > I) t.items[base + c++] = make_int2(s, I);
+    // pairs (I, I + 1) with I even, in the same order: the pairs after it are those with a
+    // larger even first row block
+    if ((I & 1) == 0) {
+      int32_t pbase = 0;
+      for (int s = 0; s < num_seqs; ++s) {
+        const int32_t e = t.nb[s] - 1 - I;
+        pbase += e > 0 ? e / 2 : 0;
+      }
+      int32_t pc = 0;
+      for (int s = 0; s < num_seqs; ++s)
+        if (t.nb[s] > I) t.pairs[pbase + pc++] = make_int2(s, I);
+    }
   }
 }
 

@@ -221,5 +221,10 @@ __device__ __forceinline__ void named_bar(uint32_t id, uint32_t threads) {
 // Host: cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
 int encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+// 3-D map {d0, d1, d2} (d0 contiguous; strides of d1 and d2 in bytes), box {b0, b1, b2},
+// 128-byte swizzle.
+int encode_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                        uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                        uint32_t b2);
 
 }  // namespace iamap
