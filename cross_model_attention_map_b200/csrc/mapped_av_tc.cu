@@ -23,10 +23,12 @@
 //     across the whole row and are written once.
 // No TMA multicast is used: every CTA loads its own tiles.
 //
-// Roles: warps 0, 8, 9, 10 load the sender slices, warp 7 builds W', warps 6 and 11 load the V
-// tiles, one thread of warp 1 issues the mixing MMAs and one thread of warp 12 the P.V MMAs (two
-// issuers: MMA and commit issue costs add up on one thread), warps 2-5 read the mixing results
-// out of TMEM, transpose and send them, and write the output. Every wait is bounded (2 s, then IAMAP_DEV_TIMEOUT).
+// Roles: warps 0, 8, 9, 10 load the sender slices, warp 7 builds W', warps 6, 11, 17, 18 load
+// the V tiles (one receiver head each), one thread of warp 1 issues the mixing MMAs and one
+// thread of warp 12 the P.V MMAs (two issuers: MMA and commit issue costs add up on one thread).
+// Two groups of four warps (2-5 and 13-16) take alternate stored blocks: they read the mixing
+// results out of TMEM, transpose and send them; the first group also writes the output. Every
+// wait is bounded (2 s, then IAMAP_DEV_TIMEOUT).
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -97,16 +99,21 @@ namespace tcav {
 
 constexpr int kG = 4;            // receiver heads per CTA (O in TMEM: 4 x 64 columns)
 constexpr int kMaxNP = 12;       // sender-slice ring: as many slots as shared memory allows
-// One warp issues TMA loads at only ~3 M per second (about 25 GB/s of 8 KB boxes, measured on
-// this B200 whatever the box layout), so the loads are spread over several producer warps: four
-// for the sender slices (chunks round-robin), two for the V tiles (receiver heads alternating),
-// and each V tile (both 64-dim halves of one head) is a single 3-D box.
-constexpr int kPWarps = 4, kVWarps = 2;
+// A thread that issues TMA loads waits ~5 ns per 128-byte line of the box (measured on this B200:
+// 0.31 us for a 16 KB contiguous box, 0.49 us for a V tile spread over 64 tokens, i.e. 33-52 GB/s
+// per issuing thread, against ~130 GB/s per SM from L2 with four issuers), so the loads are
+// spread over several producer warps: four for the sender slices (chunks round-robin) and one
+// per receiver head for the V tiles (each a single 3-D box of both 64-dim halves).
+constexpr int kPWarps = 4, kVWarps = 4;
 constexpr int kND = 8;           // mixing-result TMEM slots (chunks)
 constexpr int kNG = kND / 2;     // ... committed and released in pairs of chunks (one commit costs
                                  // ~90 ns of issue time on this B200, an MMA ~25 ns)
+constexpr int kNGh = kNG / 2;    // pair slots of each readout group: even pairs of a block use
+                                 // slots 0-1, odd pairs slots 2-3, so that every slot has one
+                                 // consumer that takes its phases in order
 constexpr int kNV = 4;           // V tiles: one slot per receiver head of the CTA
-constexpr int kThreads = 416;    // 13 warps
+constexpr int kThreads = 608;    // 19 warps
+constexpr int kEpiWarps = 8;     // two readout groups of four warps
 constexpr int kMixCol = 256;     // first TMEM column of the mixing slots
 constexpr uint32_t kTmemCols = 512;
 
@@ -199,8 +206,9 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
     // ------------------------------ sender slices (chunks round-robin over 4 warps) ------------
     const int pw = warp == 0 ? 0 : warp - 7;
     const int nch = c1 - c0;
-    int q = 0, last = -1;
+    int q = 0;
     if (lane == 0) {
+      const uint64_t pol = tc::policy_evict_first();   // each stored tile is read once
       unsigned long long m_next = T > 0 ? p.headmask[u0] : 0ull;
       int64_t off_next = T > 0 ? p.val_off[u0] : 0;
       for (int t = 0; t < T; ++t) {
@@ -219,17 +227,16 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
           if (q >= NP) tc::wait_bar(bar_addr(bars, P_EMPTY + ps), ((q / NP) - 1) & 1, abort_flag, p.status);
           tc::mbar_expect_tx(bar_addr(bars, P_FULL + ps), 2u * (uint32_t)k8 * 8u * 128u);
           const uint32_t dst = sbase + p.off_p + ps * p_stage;
-          tc::tma_load_2d(dst, &p.p_maps[k8 - 1], 0, y0 + (2 * (c0 + c)) * k, bar_addr(bars, P_FULL + ps));
-          tc::tma_load_2d(dst + p_box, &p.p_maps[k8 - 1], 0, y0 + (2 * (c0 + c) + 1) * k,
-                          bar_addr(bars, P_FULL + ps));
-          last = q;
+          tc::tma_load_2d_hint(dst, &p.p_maps[k8 - 1], 0, y0 + (2 * (c0 + c)) * k,
+                               bar_addr(bars, P_FULL + ps), pol);
+          tc::tma_load_2d_hint(dst + p_box, &p.p_maps[k8 - 1], 0, y0 + (2 * (c0 + c) + 1) * k,
+                               bar_addr(bars, P_FULL + ps), pol);
         }
       }
       // drain: the final load of every slot, where this warp issued it, has landed (earlier uses
       // of a slot are two phases back and must not be waited on)
       for (int qq = max(0, q - NP); qq < q; ++qq)
         if (qq % kPWarps == pw) tc::drain_bar(bar_addr(bars, P_FULL + qq % NP), (qq / NP) & 1);
-      (void)last;
     }
   } else if (warp == 7) {
     // ------------------------------ W' of each stored block ------------------------------
@@ -278,13 +285,14 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
       if (lane == 0) tc::mbar_arrive(bar_addr(bars, W_FULL + ws));
       __syncwarp();
     }
-  } else if (warp == 6 || warp == 11) {
-    // ------------------------------ V tiles (receiver heads alternating over 2 warps) ----------
+  } else if (warp == 6 || warp == 11 || warp == 17 || warp == 18) {
+    // ------------------------------ V tiles (one warp per receiver head) ----------------------
     // slot rl holds V_rl[J] of the current block; it is refilled once this CTA's P.V of the
     // previous block has completed (PV_DONE), so each slot is used once per block
-    const int vw = warp == 6 ? 0 : 1;
+    const int vw = warp == 6 ? 0 : warp == 11 ? 1 : warp == 17 ? 2 : 3;
     const int halves = p.d_v / 64;
     if (lane == 0) {
+      const uint64_t pol = tc::policy_evict_last();    // V_r[J] is read again by later row blocks
       int J_next = T > 0 ? p.col_idx[u0] : 0;
       for (int t = 0; t < T; ++t) {
         const int J = J_next;
@@ -292,8 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         if (t >= 1) tc::wait_bar(bar_addr(bars, PV_DONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, abort_flag, p.status);
         for (int rl = vw; rl < G; rl += kVWarps) {
           tc::mbar_expect_tx(bar_addr(bars, V_FULL + rl), v_stage);
-          tc::tma_load_3d(sbase + p.off_v + rl * v_stage, &p.v_map, 0, seq0 + J * 64,
-                          (r0 + rl) * halves, bar_addr(bars, V_FULL + rl));
+          tc::tma_load_3d_hint(sbase + p.off_v + rl * v_stage, &p.v_map, 0, seq0 + J * 64,
+                               (r0 + rl) * halves, bar_addr(bars, V_FULL + rl), pol);
         }
       }
       if (T > 0)
@@ -304,7 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
     if (lane == 0) {
       const uint32_t id_mix = tc::idesc_bf16(128, p.NR, 1, 0);
       const int nch = c1 - c0;
-      int q = 0, gq = 0;
+      const int npair = (nch + 1) >> 1;
+      int q = 0;
       int k_next = T > 0 ? __popcll(p.headmask[u0]) : 0;
       for (int t = 0; t < T; ++t) {
         const int ksteps = (k_next + 15) >> 4;
@@ -312,9 +321,12 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         const int ws = t & 1;
         tc::wait_bar(bar_addr(bars, W_FULL + ws), (t >> 1) & 1, abort_flag, p.status);
         const uint32_t wb = sbase + p.off_w + ws * w_stage;
-        for (int c = 0; c < nch; c += 2, ++gq) {
-          const int gs = gq % kNG;
-          if (gq >= kNG) tc::wait_bar(bar_addr(bars, D_EMPTY + gs), ((gq / kNG) - 1) & 1, abort_flag, p.status);
+        for (int c = 0; c < nch; c += 2) {
+          // pair lp of the block goes to readout group lp & 1, which takes its pairs in order
+          const int lp = c >> 1, g = lp & 1;
+          const int gp = t * ((npair + 1 - g) >> 1) + (lp >> 1);
+          const int gs = g * kNGh + gp % kNGh;
+          if (gp >= kNGh) tc::wait_bar(bar_addr(bars, D_EMPTY + gs), ((gp / kNGh) - 1) & 1, abort_flag, p.status);
           const int nj = min(2, nch - c);
           for (int j = 0; j < nj; ++j) {
             const int qq = q + c + j, ps = qq % NP;
@@ -367,27 +379,34 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
       tc::drain_bar(bar_addr(bars, O_FULL), 0);   // every P.V MMA completed before TMEM is freed
     }
   } else {
-    // ------------------------------ readout, exchange, output (warps 2-5) ------------------------------
+    // ------------------------------ readout, exchange, output (warps 2-5, 13-16) ----------------
+    // group eg takes the pairs lp = eg, eg + 2, ... of every block
+    const int eg = warp >= 13 ? 1 : 0;
     const int e = warp & 3;               // TMEM lane quarter of this warp
     const uint32_t lane_base = (uint32_t)(32 * e) << 16;
-    unsigned char* scr = smem + p.off_scr + (warp - 2) * 2048;   // [32 heads][32 positions] bf16
+    const int ew = eg * 4 + (warp - (eg ? 13 : 2));   // 0..7
+    unsigned char* scr = smem + p.off_scr + ew * 2048;   // [32 heads][32 positions] bf16
     const int o = lane & 3;               // this lane's 16-byte run: positions 8*o .. 8*o+7
     const int rq = lane >> 2;             // this lane's heads: 8*v + rq
     const int nch = c1 - c0;
-    int q = 0, gq = 0;
+    const int npair = (nch + 1) >> 1;
+    const bool releaser = (warp == 2 || warp == 13) && lane == 0;
+    const int npg = (npair + 1 - eg) >> 1;   // pairs of this group per block
     for (int t = 0; t < T; ++t) {
       const int ss = t & 1;
+      const int q = t * nch;          // this block's first chunk (global order)
+      int gp = t * npg;               // its first pair within this group
       // the receive buffers of round t-2 are free once every peer's P.V of that round completed
       if (t >= 2) tc::wait_bar(bar_addr(bars, BUF_FREE + ss), ((t - 2) >> 1) & 1, abort_flag, p.status);
       const uint32_t recv_local = sbase + p.off_recv + (uint32_t)ss * (kG * 8192u);
       const uint32_t rbar_local = bar_addr(bars, RECV_FULL + ss);
-      for (int cc = 0; cc < nch; ++cc) {
-        const int gs = gq % kNG, j = cc & 1;
+      for (int cc = 2 * eg; cc < nch; cc += (cc & 1) ? 3 : 1) {
+        const int gs = eg * kNGh + gp % kNGh, j = cc & 1;
         const int ch = c0 + cc;
         if (j == 0) {
-          tc::wait_bar(bar_addr(bars, D_FULL + gs), (gq / kNG) & 1, abort_flag, p.status);
+          tc::wait_bar(bar_addr(bars, D_FULL + gs), (gp / kNGh) & 1, abort_flag, p.status);
           // the pair's mixing MMAs completed: their sender slots can be refilled
-          if (warp == 2 && lane == 0)
+          if (releaser)
             for (int jj = 0; jj < min(2, nch - cc); ++jj) tc::mbar_arrive(bar_addr(bars, P_EMPTY + (q + cc + jj) % NP));
         }
         tc::tc_fence_after();
@@ -405,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
           tc::tc_fence_before();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(bar_addr(bars, D_EMPTY + gs));
-          ++gq;
+          ++gp;
         }
         // transpose: position = lane, head = register  ->  16-byte runs of one head
 #pragma unroll
@@ -429,13 +448,14 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         }
         __syncwarp();
       }
-      q += nch;
     }
-    // output rows: TMEM lane = d_v index, column = rl * 64 + row of the block
-    tc::wait_bar(bar_addr(bars, O_FULL), 0, abort_flag, p.status);
-    tc::tc_fence_after();
+    // output rows (first group): TMEM lane = d_v index, column = rl * 64 + row of the block
     const int dv = 32 * e + lane;
-    if (32 * e < p.d_v) {
+    if (eg == 0) {
+      tc::wait_bar(bar_addr(bars, O_FULL), 0, abort_flag, p.status);
+      tc::tc_fence_after();
+    }
+    if (eg == 0 && 32 * e < p.d_v) {
       for (int rl = 0; rl < G; ++rl) {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -450,9 +470,15 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         }
       }
     }
-    // the last two exchange rounds: every peer has consumed this CTA's copies and arrived here
-    for (int t = max(0, T - 2); t < T; ++t)
-      tc::wait_bar(bar_addr(bars, BUF_FREE + (t & 1)), (t >> 1) & 1, abort_flag, p.status);
+    // the last two exchange rounds: every peer's P.V commit has arrived here and every peer's copy
+    // into this CTA has landed, so nothing remote targets this CTA's shared memory once it exits.
+    // These waits ignore the abort flag (bounded at 200 ms each): after a timeout elsewhere the
+    // other threads skip their waits, and a remote arrival must still not outlive the CTA.
+    if (eg == 0)
+      for (int t = max(0, T - 2); t < T; ++t) {
+        tc::drain_bar(bar_addr(bars, BUF_FREE + (t & 1)), (t >> 1) & 1);
+        tc::drain_bar(bar_addr(bars, RECV_FULL + (t & 1)), (t >> 1) & 1);
+      }
   }
 
   tc::tc_fence_before();
@@ -485,7 +511,7 @@ int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream) {
   p.RB = (a.H_s + 7) / 8 * 8;
   // everything but the sender ring, then as many ring slots as fit (at most kMaxNP)
   const size_t fixed = (size_t)2 * p.NR * 128 + 1024 + (size_t)2 * kG * 8192 + (size_t)kNV * a.d_v * 128 +
-                       (size_t)4 * 2048 + sizeof(float) * (size_t)a.H_r * a.H_s + 8 * NUM_BARS + 96 + 4096;
+                       (size_t)kEpiWarps * 2048 + sizeof(float) * (size_t)a.H_r * a.H_s + 8 * NUM_BARS + 96 + 4096;
   const size_t p_stage_b = (size_t)2 * p.RB * 128;
   const size_t budget = 232448 - 1024;
   p.NP = (int)std::min<size_t>(kMaxNP, (budget - fixed - 1024) / p_stage_b);
@@ -502,7 +528,7 @@ int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream) {
   p.off_v = (uint32_t)off;
   off += (size_t)kNV * a.d_v * 128;
   p.off_scr = (uint32_t)off;
-  off += (size_t)4 * 2048;
+  off += (size_t)kEpiWarps * 2048;
   p.off_wf = (uint32_t)off;
   off += sizeof(float) * (size_t)a.H_r * a.H_s;
   off = round_up(off, 8);
