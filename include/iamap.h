@@ -126,9 +126,10 @@ int iamap_compress_stats(const void* q, const void* k, const int32_t* cu_seqlens
 /*
  * Compress, stage 2 (extraction of the kept blocks). Recomputes each kept (head, row block,
  * column block) tile of probabilities exp(s_ij - lse_i) from q, k and stage 1's lse, and writes
- * it as bf16 at its BSR position (row-interleaved within the block, see Layouts). A tile whose index is >= vals_capacity_tiles is not
- * written and sets IAMAP_DEV_CAPACITY in the device status. After the last tile the call also
- * zero-fills up to 64 further tiles that fit in the capacity (mapped_av may read that far).
+ * it as bf16 at its BSR position (row-interleaved within the block, see Layouts). A stored block
+ * that does not fit below vals_capacity_tiles is not written and sets IAMAP_DEV_CAPACITY in the
+ * device status. After the last tile the call also zero-fills up to 64 further tiles that fit in
+ * the capacity (mapped_av may read that far).
  */
 int iamap_compress_extract(const void* q, const void* k, const int32_t* cu_seqlens,
                            const int32_t* cu_seqlens_host, int num_seqs, int64_t n, int H_s, int d,
