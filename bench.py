@@ -55,15 +55,22 @@ CONFIG_TEXT = {
 }
 
 
+# MUFU ex2 issue rate of sm_100 (16 results per clock per SM) x 148 SMs x the maximum SM clock:
+# the ALU peak of the exp-bound statistics kernel (4.65e12 ex2/s at 1965 MHz; 4.6e12 measured).
+EX2_PER_CLK_SM = 16
+B200_SMS = 148
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
         return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
                     bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    ex2_per_s=EX2_PER_CLK_SM * B200_SMS * d.get("sm_max_mhz", 1965.0) * 1e6,
                     source="measured")
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
-                source="fallback")
+                ex2_per_s=EX2_PER_CLK_SM * B200_SMS * 1965.0e6, source="fallback")
 
 
 def src_sha(files):
@@ -303,8 +310,10 @@ def bench_prefill(args, world, rank, local, peaks):
                 + 2.0 * n * wl.H_r * wl.d_v + 4.0 * n * wl.H_r * wl.d_v + 4.0 * wl.H_r * wl.H_s)
     extract_bytes = 8192.0 * nnz_tiles + 2.0 * 2 * n * wl.H_s * wl.d + 4.0 * n * wl.H_s
     kernels = {
-        "compress_stats": {"ms": t_stats, "bound": "tensor", "flops": qk_flops,
-                           "tflops": qk_flops / (t_stats * 1e-3) / 1e12, "exps": exps},
+        "compress_stats": {"ms": t_stats, "bound": "alu", "exps": exps,
+                           "gex2_per_s": exps / (t_stats * 1e-3) / 1e9,
+                           "ex2_frac": round(exps / (t_stats * 1e-3) / peaks["ex2_per_s"], 4),
+                           "flops": qk_flops, "tflops": qk_flops / (t_stats * 1e-3) / 1e12},
         "compress_extract": {"ms": t_extract, "bound": "hbm", "bytes": extract_bytes,
                              "gbs": extract_bytes / (t_extract * 1e-3) / 1e9,
                              "tflops_qk_recompute": qk_flops * nnz_tiles / (wl.H_s * layer.ncb)
@@ -318,16 +327,22 @@ def bench_prefill(args, world, rank, local, peaks):
         achieved = kd["gbs"]
         peak = peaks["hbm_gbs"]
         unit = "GB/s"
+    elif kd["bound"] == "alu":
+        achieved = kd["gex2_per_s"]
+        peak = peaks["ex2_per_s"] / 1e9
+        unit = "Gex2/s"
     else:
         achieved = kd["tflops"]
         peak = peaks["bf16_tflops_sustained"]
         unit = "TFLOP/s"
-    files = {"mapped_av": ["mapped_av.cu"], "compress_stats": ["compress.cu", "qk_tile.cuh"],
-             "compress_extract": ["compress.cu", "qk_tile.cuh"]}[dom]
+    files = {"mapped_av": ["mapped_av_tc.cu", "tc_utils.cuh"],
+             "compress_stats": ["compress_tc.cu", "tc_utils.cuh"],
+             "compress_extract": ["compress_tc.cu", "tc_utils.cuh"]}[dom]
     roofline = {"kernel": dom, "bound": kd["bound"], "achieved": round(achieved, 2),
                 "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
                 "traffic": load_traffic(dom, files),
-                "peak_source": peaks["source"] + (" sustained bf16" if unit == "TFLOP/s" else " HBM copy")}
+                "peak_source": peaks["source"] + {"TFLOP/s": " sustained bf16", "GB/s": " HBM copy",
+                                                   "Gex2/s": " (16 ex2/clk/SM x 148 SMs x max clock)"}[unit]}
 
     # end to end through the public API with host buffers (pinned), per step: H2D of q, k, v, W,
     # cu_seqlens; the step; D2H of the output.

@@ -189,6 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
   if (warp == 8) {
     // ------------------------------ TMA: Q once, then the key tiles ------------------------------
     if (lane == 0) {
+      tc::prefetch_tmap(&p.q_map);
+      tc::prefetch_tmap(&p.k_map);
       tc::mbar_expect_tx(bar_addr(bars, Q_FULL), kQBytes);
 #pragma unroll
       for (int pan = 0; pan < NPAN; ++pan)
@@ -469,6 +471,8 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
 
   if (warp == 8) {
     if (lane == 0) {
+      tc::prefetch_tmap(&p.q_map);
+      tc::prefetch_tmap(&p.k_map);
       tc::mbar_expect_tx(bar_addr(bars, XQ_FULL), kQBytes);
 #pragma unroll
       for (int pan = 0; pan < NPAN; ++pan)

@@ -209,6 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
     int q = 0;
     if (lane == 0) {
       const uint64_t pol = tc::policy_evict_first();   // each stored tile is read once
+      if (pw == 0)
+        for (int i = 0; i < 8; ++i) tc::prefetch_tmap(&p.p_maps[i]);
       unsigned long long m_next = T > 0 ? p.headmask[u0] : 0ull;
       int64_t off_next = T > 0 ? p.val_off[u0] : 0;
       for (int t = 0; t < T; ++t) {
@@ -293,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
     const int halves = p.d_v / 64;
     if (lane == 0) {
       const uint64_t pol = tc::policy_evict_last();    // V_r[J] is read again by later row blocks
+      if (vw == 0) tc::prefetch_tmap(&p.v_map);
       int J_next = T > 0 ? p.col_idx[u0] : 0;
       for (int t = 0; t < T; ++t) {
         const int J = J_next;

@@ -113,6 +113,11 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Brings a tensor map (kernel parameter) into the TMA unit's descriptor cache.
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
 // L2 eviction policies for TMA loads: data read once (evict first) and data re-read by other
 // CTAs soon after (evict last).
 __device__ __forceinline__ uint64_t policy_evict_first() {
