@@ -80,12 +80,13 @@ def src_sha(files):
     return h.hexdigest()[:16]
 
 
-def load_traffic(kernel, files):
-    """DRAM bytes per launch from a committed ncu summary, if taken on the current source."""
+def load_traffic(kernel, workload, files):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary, if it was
+    taken on the current source; else None."""
     p = os.path.join(PROFILES, "dram_traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get(kernel)
+    d = json.load(open(p)).get(kernel, {}).get(workload)
     if not d or d.get("source_sha") != src_sha(files):
         return None
     return d.get("bytes_per_launch")
@@ -340,7 +341,7 @@ def bench_prefill(args, world, rank, local, peaks):
              "compress_extract": ["compress_tc.cu", "tc_utils.cuh"]}[dom]
     roofline = {"kernel": dom, "bound": kd["bound"], "achieved": round(achieved, 2),
                 "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
-                "traffic": load_traffic(dom, files),
+                "traffic": load_traffic(dom, args.config, files),
                 "peak_source": peaks["source"] + {"TFLOP/s": " sustained bf16", "GB/s": " HBM copy",
                                                    "Gex2/s": " (16 ex2/clk/SM x 148 SMs x max clock)"}[unit]}
 
@@ -439,7 +440,7 @@ def bench_decode(args, world, rank, local, peaks):
         "roofline": {"kernel": "paged_gemv", "bound": "hbm", "achieved": round(gbs, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gbs / peaks["hbm_gbs"], 4),
-                     "traffic": load_traffic("paged_gemv", ["decode.cu"])},
+                     "traffic": load_traffic("paged_gemv", "decode", ["decode.cu"])},
         "clocks": clocks, "gpu_launches": 2 * args.steps,
     }, dw
 

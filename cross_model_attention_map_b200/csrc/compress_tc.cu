@@ -138,6 +138,47 @@ __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
+// c = log2 of sum_j 2^(x_j) over one thread's 64 logits of column block J (keys j0 .. j0 + 63) of
+// row i, x_j = s_j * sc (+ bias_log2 where 0 <= i - j < bias_window), x_j = -inf above the
+// diagonal. `plain`: J is below the row's block, so there is no mask, and the bias is checked.
+// The masked path overwrites v with the x_j.
+__device__ __forceinline__ float block_log2sum(uint32_t (&v)[64], int i, int j0, bool plain,
+                                               float sc, int bias_window, float bias_log2) {
+  if (plain && !(bias_window > 0 && i - j0 - 63 < bias_window)) {
+    float m8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(v[k]);
+#pragma unroll
+    for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
+    const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+    const float nm = -mx * sc;
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < 64; ++e) s4[e & 3] += ex2(fmaf(__uint_as_float(v[e]), sc, nm));
+    return mx * sc + lg2((s4[0] + s4[1]) + (s4[2] + s4[3]));
+  }
+  float m8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < 64; ++e) {
+    const int j = j0 + e;
+    float y = __uint_as_float(v[e]) * sc;
+    if (bias_window > 0 && i - j >= 0 && i - j < bias_window) y += bias_log2;
+    y = j > i ? -INFINITY : y;
+    v[e] = __float_as_uint(y);
+    m8[e & 7] = fmaxf(m8[e & 7], y);
+  }
+  const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+  if (mx == -INFINITY) return -INFINITY;
+  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int e = 0; e < 64; ++e) s4[e & 3] += ex2(__uint_as_float(v[e]) - mx);
+  return mx + lg2((s4[0] + s4[1]) + (s4[2] + s4[3]));
+}
+
 // ------------------------------------------------------------------------------------------------
 // Stage 1: block statistics, masses and the per-head choice
 // ------------------------------------------------------------------------------------------------
@@ -242,68 +283,52 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
     const uint32_t t_lane = (uint32_t)(32 * qd) << 16;
     const float sc = p.scale_log2;
     float m_acc = -INFINITY, l_acc = 0.f;
-    for (int T = 0; T < nT; ++T) {
-      const int b = T & 1;
-      const int J = 2 * T + g;
-      tc::wait_bar(bar_addr(bars, S_FULL + b), (T >> 1) & 1, abort_flag, p.status);
-      tc::tc_fence_after();
-      uint32_t v[64];
-      if (J <= Ir) {
-        IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(b * 128 + g * 64), v);
-        IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(b * 128 + g * 64 + 32), (v + 32));
-        tc::tmem_ld_wait();
+    // The TMEM load of tile T + 1 is issued before the exponentials of tile T, so that its latency
+    // hides behind them (two register sets, the loop unrolled by two).
+    uint32_t va[64], vb[64];
+    auto issue = [&](uint32_t (&v)[64], int T) {
+      if (2 * T + g <= Ir) {
+        const uint32_t col = (uint32_t)((T & 1) * 128 + g * 64);
+        IAMAP_TMEM_LD32(tmem + t_lane + col, v);
+        IAMAP_TMEM_LD32(tmem + t_lane + col + 32u, (v + 32));
       }
+    };
+    auto step = [&](uint32_t (&cur)[64], uint32_t (&nxt)[64], int T) {
+      const int J = 2 * T + g;
+      if (J <= Ir) tc::tmem_ld_wait();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar_addr(bars, S_EMPTY + b));
-      if (J > Ir) continue;
-      const int j0 = 64 * J;
-      float c;
-      if (J < Ir && !(p.bias_window > 0 && i - j0 - 63 < p.bias_window)) {
-        // no causal mask and no bias inside this block
-        float mx = __uint_as_float(v[0]);
-#pragma unroll
-        for (int e = 1; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
-        const float nm = -mx * sc;
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-        for (int e = 0; e < 64; e += 4) {
-          s0 += ex2(fmaf(__uint_as_float(v[e]), sc, nm));
-          s1 += ex2(fmaf(__uint_as_float(v[e + 1]), sc, nm));
-          s2 += ex2(fmaf(__uint_as_float(v[e + 2]), sc, nm));
-          s3 += ex2(fmaf(__uint_as_float(v[e + 3]), sc, nm));
-        }
-        c = mx * sc + lg2((s0 + s1) + (s2 + s3));
-      } else {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const int j = j0 + e;
-          float x = __uint_as_float(v[e]) * sc;
-          if (p.bias_window > 0 && i - j >= 0 && i - j < p.bias_window) x += p.bias_log2;
-          x = j > i ? -INFINITY : x;
-          v[e] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
-        if (mx == -INFINITY) {
-          c = -INFINITY;
-        } else {
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            s0 += ex2(__uint_as_float(v[e]) - mx);
-            s1 += ex2(__uint_as_float(v[e + 1]) - mx);
-          }
-          c = mx + lg2(s0 + s1);
-        }
+      if (lane == 0) tc::mbar_arrive(bar_addr(bars, S_EMPTY + (T & 1)));
+      bool early = false;
+      if (T + 1 < nT && tc::mbar_try_wait(bar_addr(bars, S_FULL + ((T + 1) & 1)), ((T + 1) >> 1) & 1)) {
+        tc::tc_fence_after();
+        issue(nxt, T + 1);
+        early = true;
       }
-      if (c > m_acc) {
-        l_acc = l_acc * ex2(m_acc - c) + 1.f;
-        m_acc = c;
-      } else if (c > -INFINITY) {
-        l_acc += ex2(c - m_acc);
+      if (J <= Ir) {
+        const float c = block_log2sum(cur, i, 64 * J, J < Ir, sc, p.bias_window, p.bias_log2);
+        if (c > m_acc) {
+          l_acc = l_acc * ex2(m_acc - c) + 1.f;
+          m_acc = c;
+        } else if (c > -INFINITY) {
+          l_acc += ex2(c - m_acc);
+        }
+        tmem_st1(tmem + t_lane + (uint32_t)(kCCol + J), c);
       }
-      tmem_st1(tmem + t_lane + (uint32_t)(kCCol + J), c);
+      if (T + 1 < nT && !early) {
+        tc::wait_bar(bar_addr(bars, S_FULL + ((T + 1) & 1)), ((T + 1) >> 1) & 1, abort_flag, p.status);
+        tc::tc_fence_after();
+        issue(nxt, T + 1);
+      }
+    };
+    if (nT > 0) {
+      tc::wait_bar(bar_addr(bars, S_FULL), 0, abort_flag, p.status);
+      tc::tc_fence_after();
+      issue(va, 0);
+    }
+    for (int T = 0; T < nT; T += 2) {
+      step(va, vb, T);
+      if (T + 1 < nT) step(vb, va, T + 1);
     }
     tmem_st_wait();
 
@@ -541,18 +566,19 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
         // the row at c ^ (row & 7))
         const int j0 = 64 * J;
         const bool fast = J < Ir && !(p.bias_window > 0 && i - j0 - 63 < p.bias_window);
+        uint32_t v[64];
+        IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(b * 64), v);
+        IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(b * 64 + 32), (v + 32));
+        tc::tmem_ld_wait();
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t v[32];
-          IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(b * 64 + 32 * half), v);
-          tc::tmem_ld_wait();
           uint32_t pk[16];
           if (fast) {
             const float nl = -lse2;
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-              const float a0 = valid ? ex2(fmaf(__uint_as_float(v[e]), sc, nl)) : 0.f;
-              const float a1 = valid ? ex2(fmaf(__uint_as_float(v[e + 1]), sc, nl)) : 0.f;
+              const float a0 = valid ? ex2(fmaf(__uint_as_float(v[32 * half + e]), sc, nl)) : 0.f;
+              const float a1 = valid ? ex2(fmaf(__uint_as_float(v[32 * half + e + 1]), sc, nl)) : 0.f;
               pk[e >> 1] = pack_bf16(a0, a1);
             }
           } else {
@@ -562,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
 #pragma unroll
               for (int u = 0; u < 2; ++u) {
                 const int j = j0 + 32 * half + e + u;
-                float x = __uint_as_float(v[e + u]) * sc;
+                float x = __uint_as_float(v[32 * half + e + u]) * sc;
                 if (p.bias_window > 0 && i - j >= 0 && i - j < p.bias_window) x += p.bias_log2;
                 a[u] = (valid && j <= i) ? ex2(x - lse2) : 0.f;
               }
