@@ -8,9 +8,12 @@
 //
 // The V cache stream dominates (bytes read once), so the kernel is a coalesced GEMV on CUDA
 // cores: CTA (chunk of pages, sequence b, slice of 8192 output elements) walks its pages; each
-// thread owns four 16-byte chunks of the [H_r * d_v] token row and accumulates fp32. The mixed
-// weights of the page's tokens are formed in shared memory first. Partial sums per page chunk go
-// to the workspace and a second kernel adds them in a fixed order (deterministic).
+// thread owns four 16-byte chunks of the [H_r * d_v] token row and accumulates fp32, with the
+// loads of four tokens in flight. The mixed weights of up to 128 tokens are formed in shared
+// memory at a time. Partial sums per page chunk go to the workspace and a second kernel adds them
+// in a fixed order (deterministic).
+#include <algorithm>
+
 #include "internal.h"
 
 namespace iamap {
@@ -37,9 +40,13 @@ struct DecParams {
   unsigned int* status;
 };
 
-__global__ void __launch_bounds__(kDecThreads) paged_gemv_kernel(DecParams p) {
-  __shared__ float s_p[kDecMaxPage * kDecMaxH];    // [slot][s] sender probabilities
-  __shared__ float s_w[kDecMaxPage * kDecMaxH];    // [slot][r] mixed weights
+// Mixed weights of kDecGroupTok tokens are formed at a time in shared memory:
+// s_w[t][r] = sum_s W[r, s] p[b, s, j0 + t] (W read through L1).
+constexpr int kDecGroupTok = 128;
+constexpr int kDecUnroll = 3;                               // tokens whose loads are in flight
+
+__global__ void __launch_bounds__(kDecThreads, 2) paged_gemv_kernel(DecParams p) {
+  extern __shared__ float s_w[];                   // [kDecGroupTok][H_r]
   const int chunk = blockIdx.x, b = blockIdx.y, slice = blockIdx.z;
   const int tid = threadIdx.x;
   const int E = p.H_r * p.d_v;
@@ -47,6 +54,7 @@ __global__ void __launch_bounds__(kDecThreads) paged_gemv_kernel(DecParams p) {
   const int npages = (ctx + p.page_size - 1) / p.page_size;
   const int pg0 = chunk * p.ppc, pg1 = min(npages, pg0 + p.ppc);
   const int e0 = slice * kDecSlice;
+  const int gpages = max(1, kDecGroupTok / p.page_size);    // pages per weight group
 
   float acc[kDecCPT][8];
 #pragma unroll
@@ -63,45 +71,52 @@ __global__ void __launch_bounds__(kDecThreads) paged_gemv_kernel(DecParams p) {
   }
   const float* prow = p.p_rows + (int64_t)b * p.H_s * p.ctx_stride;
   bool bad = false;
-  for (int pi = pg0; pi < pg1; ++pi) {
-    const int j0 = pi * p.page_size;
-    const int nslot = min(p.page_size, ctx - j0);
-    __syncthreads();
-    for (int e = tid; e < p.page_size * p.H_s; e += kDecThreads) {
-      const int t = e / p.H_s, sh = e % p.H_s;
-      s_p[t * kDecMaxH + sh] = t < nslot ? prow[(int64_t)sh * p.ctx_stride + j0 + t] : 0.f;
-    }
-    __syncthreads();
-    for (int e = tid; e < p.page_size * p.H_r; e += kDecThreads) {
-      const int t = e / p.H_r, r = e % p.H_r;
+  for (int gp0 = pg0; gp0 < pg1; gp0 += gpages) {
+    const int gp1 = min(pg1, gp0 + gpages);
+    const int j0 = gp0 * p.page_size;
+    const int ntok = min(ctx, gp1 * p.page_size) - j0;
+    __syncthreads();   // the previous group's weights are no longer read
+    for (int e = tid; e < ntok * p.H_r; e += kDecThreads) {
+      const int r = e / ntok, t = e - r * ntok;       // consecutive threads: consecutive tokens
       float w = 0.f;
-      for (int sh = 0; sh < p.H_s; ++sh) w = fmaf(p.W[r * p.H_s + sh], s_p[t * kDecMaxH + sh], w);
-      s_w[t * kDecMaxH + r] = w;
+      for (int sh = 0; sh < p.H_s; ++sh)
+        w = fmaf(__ldg(p.W + r * p.H_s + sh), __ldg(prow + (int64_t)sh * p.ctx_stride + j0 + t), w);
+      s_w[t * p.H_r + r] = w;
     }
     __syncthreads();
-    const int pg = p.page_table[(int64_t)b * p.max_pages + pi];
-    if (pg < 0 || pg >= p.num_pages) {
-      bad = true;
-      continue;
-    }
-    const __nv_bfloat16* vpage = p.v + (int64_t)pg * p.page_size * E;
-    for (int t = 0; t < nslot; ++t) {
-      uint4 raw[kDecCPT];
+    for (int pi = gp0; pi < gp1; ++pi) {
+      const int pg = p.page_table[(int64_t)b * p.max_pages + pi];
+      if (pg < 0 || pg >= p.num_pages) {
+        bad = true;
+        continue;
+      }
+      const int tb = (pi - gp0) * p.page_size;          // first token of the page in the group
+      const int nslot = min(p.page_size, ctx - pi * p.page_size);
+      const __nv_bfloat16* vpage = p.v + (int64_t)pg * p.page_size * E;
+      for (int t0 = 0; t0 < nslot; t0 += kDecUnroll) {
+        uint4 raw[kDecUnroll][kDecCPT];
 #pragma unroll
-      for (int c = 0; c < kDecCPT; ++c)
-        if (live[c])
-          raw[c] = __ldg(reinterpret_cast<const uint4*>(vpage + (int64_t)t * E + e0 +
-                                                        (c * kDecThreads + tid) * 8));
+        for (int u = 0; u < kDecUnroll; ++u)
 #pragma unroll
-      for (int c = 0; c < kDecCPT; ++c) {
-        if (!live[c]) continue;
-        const float w = s_w[t * kDecMaxH + head_of[c]];
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[c]);
+          for (int c = 0; c < kDecCPT; ++c)
+            if (live[c] && t0 + u < nslot)
+              raw[u][c] = __ldg(reinterpret_cast<const uint4*>(
+                  vpage + (int64_t)(t0 + u) * E + e0 + (c * kDecThreads + tid) * 8));
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(h2[e]);
-          acc[c][2 * e] = fmaf(w, f.x, acc[c][2 * e]);
-          acc[c][2 * e + 1] = fmaf(w, f.y, acc[c][2 * e + 1]);
+        for (int u = 0; u < kDecUnroll; ++u) {
+          if (t0 + u >= nslot) break;
+#pragma unroll
+          for (int c = 0; c < kDecCPT; ++c) {
+            if (!live[c]) continue;
+            const float w = s_w[(tb + t0 + u) * p.H_r + head_of[c]];
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u][c]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h2[e]);
+              acc[c][2 * e] = fmaf(w, f.x, acc[c][2 * e]);
+              acc[c][2 * e + 1] = fmaf(w, f.y, acc[c][2 * e + 1]);
+            }
+          }
         }
       }
     }
@@ -170,7 +185,11 @@ int mapped_av_paged_impl(const PagedArgs& a, cudaStream_t stream) {
   p.status = a.status;
   const int E = a.H_r * a.d_v;
   dim3 grid(a.chunks, a.batch, (E + kDecSlice - 1) / kDecSlice);
-  paged_gemv_kernel<<<grid, kDecThreads, 0, stream>>>(p);
+  const int gtok = std::max(1, kDecGroupTok / a.page_size) * a.page_size;
+  const size_t smem = sizeof(float) * (size_t)gtok * a.H_r;
+  IAMAP_CUDA_CHECK(cudaFuncSetAttribute(paged_gemv_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  paged_gemv_kernel<<<grid, kDecThreads, smem, stream>>>(p);
   IAMAP_LAUNCH_CHECK("paged_gemv_kernel");
   dim3 rgrid((E / 4 + 255) / 256, a.batch);
   paged_reduce_kernel<<<rgrid, 256, 0, stream>>>(a.partial, a.chunks, E, a.out);
