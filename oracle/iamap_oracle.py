@@ -59,7 +59,7 @@ __all__ = [
     "NEAR_EPS", "CausalLayout", "causal_layout", "head_rows", "scores", "softmax_rows",
     "block_masses", "select_blocks", "RowBlockStats", "rowblock_stats", "CompressResult",
     "compress", "union_bsr", "masked_tile", "mapped_av_rows", "mapped_av", "mapped_av_paged",
-    "attention_map", "head_match",
+    "attention_map", "head_match", "mapping_consistency",
 ]
 
 
@@ -351,22 +351,34 @@ def attention_map(q: np.ndarray, k: np.ndarray) -> np.ndarray:
     return p
 
 
-def head_match(hm, n_used=None):
-    """Cosine similarity of flattened causal maps of every large head with every small head, and
-    the most similar small head per large head (ties: lowest index).
+def head_match(hm, n_used=None, metric="cosine"):
+    """Similarity of the flattened causal maps of every large head with every small head, and
+    the most similar small head per large head (ties: lowest index). IAM notes, method section 1
+    (flatten the attention matrices, compare with cosine similarity, Minkowski distance or the
+    Pearson correlation) and section 4 (for each head of a mapped large layer, the most similar
+    small head; prompts longer than tau_t are truncated).
+
+    metric: "cosine" (a.b / |a||b|), "pearson" (the correlation coefficient of the n*n entries of
+    the two maps: the cosine of the maps less their means) or "euclidean" (the Minkowski distance
+    with p = 2, negated so that the largest value is the most similar head).
 
     Small heads are indexed layer-major (layer * H_small + head), large heads likewise. Truncation
-    to the first n_used tokens (tau_t) uses the maps of that prefix. Returns (C [L_l*H_large,
+    to the first n_used tokens (tau_t) uses the maps of that prefix. Returns (S [L_l*H_large,
     L_s*H_small], argmax int32 [L_l, H_large])."""
     n = hm.n if n_used is None else int(n_used)
     ns = hm.L_s * hm.H_small
-    small = np.zeros((ns, n * n))
-    for l in range(hm.L_s):
-        for h in range(hm.H_small):
-            A = attention_map(bf16_bits_to_f64(hm.q_small[l, :n, h]),
-                              bf16_bits_to_f64(hm.k_small[l, :n, h]))
-            small[l * hm.H_small + h] = A.ravel()
-    small_norm = np.sqrt(np.sum(small * small, axis=1))
+
+    def flat_maps(q, k, layers, heads):
+        out = np.zeros((layers * heads, n * n))
+        for l in range(layers):
+            for h in range(heads):
+                A = attention_map(bf16_bits_to_f64(q[l, :n, h]), bf16_bits_to_f64(k[l, :n, h]))
+                out[l * heads + h] = A.ravel()
+        return out
+
+    small = flat_maps(hm.q_small, hm.k_small, hm.L_s, hm.H_small)
+    if metric == "pearson":
+        small = small - small.mean(axis=1, keepdims=True)
     C = np.zeros((hm.L_l * hm.H_large, ns))
     for l in range(hm.L_l):
         large = np.zeros((hm.H_large, n * n))
@@ -374,8 +386,24 @@ def head_match(hm, n_used=None):
             A = attention_map(bf16_bits_to_f64(hm.q_large[l, :n, h]),
                               bf16_bits_to_f64(hm.k_large[l, :n, h]))
             large[h] = A.ravel()
-        large_norm = np.sqrt(np.sum(large * large, axis=1))
-        C[l * hm.H_large:(l + 1) * hm.H_large] = (large @ small.T) / (
-            large_norm[:, None] * small_norm[None, :])
+        rows = slice(l * hm.H_large, (l + 1) * hm.H_large)
+        if metric in ("cosine", "pearson"):
+            if metric == "pearson":
+                large = large - large.mean(axis=1, keepdims=True)
+            C[rows] = (large @ small.T) / (np.linalg.norm(large, axis=1)[:, None]
+                                           * np.linalg.norm(small, axis=1)[None, :])
+        elif metric == "euclidean":
+            for h in range(hm.H_large):
+                C[l * hm.H_large + h] = -np.linalg.norm(small - large[h][None, :], axis=1)
+        else:
+            raise ValueError("unknown metric %r" % (metric,))
     arg = np.argmax(C, axis=1).astype(np.int32).reshape(hm.L_l, hm.H_large)
     return C, arg
+
+
+def mapping_consistency(a, b) -> float:
+    """Share of large heads that two head mappings send to the same small head (IAM notes,
+    method section 3: the mapping built at prefill stays consistent during decode)."""
+    a = np.asarray(a).ravel()
+    b = np.asarray(b).ravel()
+    return float(np.mean(a == b))

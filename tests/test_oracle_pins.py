@@ -348,6 +348,61 @@ def test_head_match_cosine_equals_sklearn():
                                rtol=1e-12, atol=1e-14)
 
 
+def _flat_maps(hm, q, k, layers, heads, n):
+    return np.array([O.attention_map(bf16_bits_to_f64(q[l, :n, h]),
+                                     bf16_bits_to_f64(k[l, :n, h])).ravel()
+                     for l in range(layers) for h in range(heads)])
+
+
+def test_head_match_pearson_equals_scipy():
+    """Pearson metric = scipy.stats.pearsonr of the flattened n x n maps, pair by pair."""
+    from scipy.stats import pearsonr
+    hm = make_head_match(n=40, L_s=2, H_small=3, d_small=8, L_l=1, H_large=4, d_large=16,
+                         noise=0.5, seed=17)
+    S, arg = O.head_match(hm, metric="pearson")
+    small = _flat_maps(hm, hm.q_small, hm.k_small, 2, 3, 40)
+    large = _flat_maps(hm, hm.q_large, hm.k_large, 1, 4, 40)
+    ref = np.array([[pearsonr(a, b)[0] for b in small] for a in large])
+    np.testing.assert_allclose(S, ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_array_equal(arg.ravel(), np.argmax(ref, axis=1))
+    # every causal softmax row sums to 1, so every map's mean is 1/n
+    np.testing.assert_allclose(small.mean(axis=1), 1.0 / 40, rtol=1e-12)
+
+
+def test_head_match_euclidean_equals_scipy_cdist():
+    """Euclidean metric = minus scipy's Minkowski (p = 2) distance of the flattened maps, also
+    on a truncated prefix."""
+    from scipy.spatial.distance import cdist
+    hm = make_head_match(n=36, L_s=1, H_small=5, d_small=8, L_l=2, H_large=3, d_large=8,
+                         noise=0.4, seed=18)
+    for n_used in (36, 17):
+        S, arg = O.head_match(hm, n_used=n_used, metric="euclidean")
+        small = _flat_maps(hm, hm.q_small, hm.k_small, 1, 5, n_used)
+        large = _flat_maps(hm, hm.q_large, hm.k_large, 2, 3, n_used)
+        ref = -cdist(large, small, metric="minkowski", p=2)
+        np.testing.assert_allclose(S, ref, rtol=1e-10, atol=1e-13)
+        np.testing.assert_array_equal(arg.ravel(), np.argmax(ref, axis=1))
+
+
+def test_head_match_metrics_agree_on_exact_copies():
+    """Noise-free copies with equal head dims: every metric picks the planted head (cosine and
+    Pearson 1, distance 0)."""
+    hm = make_head_match(n=32, L_s=2, H_small=3, d_small=8, L_l=1, H_large=5, d_large=8,
+                         noise=0.0, seed=19)
+    for metric, best in (("cosine", 1.0), ("pearson", 1.0), ("euclidean", 0.0)):
+        S, arg = O.head_match(hm, metric=metric)
+        np.testing.assert_array_equal(arg, hm.planted)
+        for h in range(5):
+            assert abs(S[h, hm.planted[0, h]] - best) < 1e-10
+
+
+def test_mapping_consistency_counts_equal_entries():
+    a = np.array([3, 1, 4, 1, 5, 9, 2, 6], dtype=np.int32)
+    b = np.array([3, 1, 4, 0, 5, 8, 2, 6], dtype=np.int32)
+    assert O.mapping_consistency(a, b) == 6 / 8
+    assert O.mapping_consistency(a, a) == 1.0
+
+
 def test_head_match_exact_copy_has_cosine_one():
     hm = make_head_match(n=32, L_s=2, H_small=3, d_small=8, L_l=1, H_large=5, d_large=8,
                          noise=0.0, seed=16)
