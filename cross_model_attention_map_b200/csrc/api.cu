@@ -168,10 +168,24 @@ extern "C" int iamap_mapped_av(const int32_t* cu_seqlens, const int32_t* cu_seql
                                int64_t vals_capacity_tiles, const float* W, int H_r,
                                const void* v, int d_v, float* out, void* ws, size_t ws_bytes,
                                void* stream) {
+  return iamap_mapped_av_gqa(cu_seqlens, cu_seqlens_host, num_seqs, n, B, H_s, row_ptr, col_idx,
+                             headmask, val_off, vals, vals_capacity_tiles, W, H_r, H_r, v, d_v,
+                             out, ws, ws_bytes, stream);
+}
+
+extern "C" int iamap_mapped_av_gqa(const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                                   int num_seqs, int64_t n, int B, int H_s, const int32_t* row_ptr,
+                                   const int32_t* col_idx, const uint64_t* headmask,
+                                   const int64_t* val_off, const void* vals,
+                                   int64_t vals_capacity_tiles, const float* W, int H_r, int H_kv,
+                                   const void* v, int d_v, float* out, void* ws, size_t ws_bytes,
+                                   void* stream) {
   clear_error();
   int rc = check_common(B, H_s, d_v);
   if (rc) return rc;
   if (H_r < 1) return set_error(IAMAP_ERR_INVALID_ARG, "H_r must be >= 1");
+  if (H_kv < 1 || H_r % H_kv != 0)
+    return set_error(IAMAP_ERR_INVALID_ARG, "H_kv=%d must divide H_r=%d", H_kv, H_r);
   if (!row_ptr || !col_idx || !headmask || !val_off || !W || !v || !out ||
       (!vals && vals_capacity_tiles > 0))
     return set_error(IAMAP_ERR_INVALID_ARG, "null tensor pointer");
@@ -196,6 +210,7 @@ extern "C" int iamap_mapped_av(const int32_t* cu_seqlens, const int32_t* cu_seql
   a.capacity = vals_capacity_tiles;
   a.W = W;
   a.H_r = H_r;
+  a.H_kv = H_kv;
   a.v = v;
   a.d_v = d_v;
   a.out = out;
@@ -219,7 +234,20 @@ extern "C" int iamap_mapped_av_paged(const float* p_rows, int ctx_stride, const 
                                      const int32_t* ctx_lens, const int32_t* ctx_lens_host,
                                      int batch, int H_s, int H_r, int d_v, float* out, void* ws,
                                      size_t ws_bytes, void* stream) {
+  return iamap_mapped_av_paged_gqa(p_rows, ctx_stride, W, v_pages, num_pages, page_table,
+                                   max_pages, page_size, ctx_lens, ctx_lens_host, batch, H_s, H_r,
+                                   H_r, d_v, out, ws, ws_bytes, stream);
+}
+
+extern "C" int iamap_mapped_av_paged_gqa(const float* p_rows, int ctx_stride, const float* W,
+                                         const void* v_pages, int64_t num_pages,
+                                         const int32_t* page_table, int max_pages, int page_size,
+                                         const int32_t* ctx_lens, const int32_t* ctx_lens_host,
+                                         int batch, int H_s, int H_r, int H_kv, int d_v,
+                                         float* out, void* ws, size_t ws_bytes, void* stream) {
   clear_error();
+  if (H_kv < 1 || H_r < 1 || H_r % H_kv != 0)
+    return set_error(IAMAP_ERR_INVALID_ARG, "H_kv=%d must divide H_r=%d", H_kv, H_r);
   if (!p_rows || !W || !v_pages || !page_table || !ctx_lens || !ctx_lens_host || !out)
     return set_error(IAMAP_ERR_INVALID_ARG, "null pointer");
   if (batch < 1 || H_s < 1 || H_r < 1 || page_size < 1 || max_pages < 0 || num_pages < 0)
@@ -253,6 +281,7 @@ extern "C" int iamap_mapped_av_paged(const float* p_rows, int ctx_stride, const 
   a.ctx_lens = ctx_lens;
   a.max_ctx = max_ctx;
   a.batch = batch;
+  a.H_kv = H_kv;
   a.H_s = H_s;
   a.H_r = H_r;
   a.d_v = d_v;
@@ -272,7 +301,28 @@ extern "C" int iamap_head_match(const void* q_small, const void* k_small, int L_
                                 int d_small, const void* q_large, const void* k_large, int L_l,
                                 int H_large, int d_large, int n, int n_used, int32_t* argmax,
                                 float* sim, void* ws, size_t ws_bytes, void* stream) {
+  return iamap_head_match_metric(q_small, k_small, L_s, H_small, d_small, q_large, k_large, L_l,
+                                 H_large, d_large, n, n_used, IAMAP_SIM_COSINE, argmax, sim, ws,
+                                 ws_bytes, stream);
+}
+
+extern "C" int iamap_mapping_consistency(const int32_t* a, const int32_t* b, int n_heads,
+                                         int32_t* agree, void* stream) {
   clear_error();
+  if (!a || !b || !agree) return set_error(IAMAP_ERR_INVALID_ARG, "null pointer");
+  if (n_heads < 1) return set_error(IAMAP_ERR_INVALID_ARG, "n_heads must be >= 1");
+  if (!device_context()) return IAMAP_ERR_CUDA;
+  return consistency_impl(a, b, n_heads, agree, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int iamap_head_match_metric(const void* q_small, const void* k_small, int L_s,
+                                       int H_small, int d_small, const void* q_large,
+                                       const void* k_large, int L_l, int H_large, int d_large,
+                                       int n, int n_used, int metric, int32_t* argmax, float* sim,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (metric != IAMAP_SIM_COSINE && metric != IAMAP_SIM_PEARSON && metric != IAMAP_SIM_EUCLIDEAN)
+    return set_error(IAMAP_ERR_INVALID_ARG, "unknown similarity metric %d", metric);
   if (!q_small || !k_small || !q_large || !k_large || !argmax)
     return set_error(IAMAP_ERR_INVALID_ARG, "null pointer");
   if (L_s < 1 || H_small < 1 || L_l < 1 || H_large < 1 || n < 1 || n_used < 1 || n_used > n)
@@ -301,6 +351,7 @@ extern "C" int iamap_head_match(const void* q_small, const void* k_small, int L_
   a.d_large = d_large;
   a.n = n;
   a.n_used = n_used;
+  a.metric = metric;
   a.argmax = argmax;
   a.sim = sim;
   a.ws = ws;

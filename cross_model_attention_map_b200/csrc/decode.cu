@@ -35,6 +35,7 @@ struct DecParams {
   int page_size;
   const int32_t* ctx_lens;
   int H_s, H_r, d_v;
+  int kv_grp;   // receiver heads per value head
   int chunks, ppc;
   float* partial;
   unsigned int* status;
@@ -49,7 +50,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) paged_gemv_kernel(DecParams p)
   extern __shared__ float s_w[];                   // [kDecGroupTok][H_r]
   const int chunk = blockIdx.x, b = blockIdx.y, slice = blockIdx.z;
   const int tid = threadIdx.x;
-  const int E = p.H_r * p.d_v;
+  const int E = p.H_r * p.d_v;                    // output elements per sequence
+  const int Ev = (p.H_r / p.kv_grp) * p.d_v;      // value elements per token
   const int ctx = p.ctx_lens[b];
   const int npages = (ctx + p.page_size - 1) / p.page_size;
   const int pg0 = chunk * p.ppc, pg1 = min(npages, pg0 + p.ppc);
@@ -62,12 +64,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) paged_gemv_kernel(DecParams p)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[c][e] = 0.f;
   int head_of[kDecCPT];
+  int voff[kDecCPT];   // element offset of this chunk in a token's value row
   bool live[kDecCPT];
 #pragma unroll
   for (int c = 0; c < kDecCPT; ++c) {
     const int e = e0 + (c * kDecThreads + tid) * 8;
     live[c] = e < E;
     head_of[c] = live[c] ? e / p.d_v : 0;
+    voff[c] = live[c] ? (head_of[c] / p.kv_grp) * p.d_v + (e - head_of[c] * p.d_v) : 0;
   }
   const float* prow = p.p_rows + (int64_t)b * p.H_s * p.ctx_stride;
   bool bad = false;
@@ -92,7 +96,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) paged_gemv_kernel(DecParams p)
       }
       const int tb = (pi - gp0) * p.page_size;          // first token of the page in the group
       const int nslot = min(p.page_size, ctx - pi * p.page_size);
-      const __nv_bfloat16* vpage = p.v + (int64_t)pg * p.page_size * E;
+      const __nv_bfloat16* vpage = p.v + (int64_t)pg * p.page_size * Ev;
       for (int t0 = 0; t0 < nslot; t0 += kDecUnroll) {
         uint4 raw[kDecUnroll][kDecCPT];
 #pragma unroll
@@ -100,8 +104,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) paged_gemv_kernel(DecParams p)
 #pragma unroll
           for (int c = 0; c < kDecCPT; ++c)
             if (live[c] && t0 + u < nslot)
-              raw[u][c] = __ldg(reinterpret_cast<const uint4*>(
-                  vpage + (int64_t)(t0 + u) * E + e0 + (c * kDecThreads + tid) * 8));
+              raw[u][c] = __ldg(reinterpret_cast<const uint4*>(vpage + (int64_t)(t0 + u) * Ev + voff[c]));
 #pragma unroll
         for (int u = 0; u < kDecUnroll; ++u) {
           if (t0 + u >= nslot) break;
@@ -179,6 +182,7 @@ int mapped_av_paged_impl(const PagedArgs& a, cudaStream_t stream) {
   p.H_s = a.H_s;
   p.H_r = a.H_r;
   p.d_v = a.d_v;
+  p.kv_grp = a.H_r / (a.H_kv > 0 ? a.H_kv : a.H_r);
   p.chunks = a.chunks;
   p.ppc = a.pages_per_chunk;
   p.partial = a.partial;

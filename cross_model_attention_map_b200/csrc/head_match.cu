@@ -10,8 +10,14 @@
 //    accumulated alongside.
 // 2. gram_kernel: C_raw = A_large . A_small^T over the flattened maps (split-K, mma.sync,
 //    fp32 accumulate, atomic fp32 reduction of the K splits).
-// 3. finalize_kernel: cosine = C_raw / (|A_large| |A_small|) and the argmax per large head
-//    (lowest small-head index on ties).
+// 3. finalize_kernel: the similarity of every (large, small) pair from C_raw and each map's sum and
+//    squared norm, and the argmax per large head (lowest small-head index on ties). The method
+//    section of the IAM notes compares cosine similarity, Minkowski distance and the Pearson
+//    correlation of the flattened maps: cosine = C / (|a| |b|); Pearson = the cosine of the
+//    maps less their means over the n_used x n_used entries; Minkowski with p = 2 (Euclidean):
+//    |a - b|^2 = |a|^2 + |b|^2 - 2 C, reported negated so that larger is more similar.
+// 4. consistency_kernel: how many large heads two mappings (e.g. prefill and a later prefix)
+//    send to the same small head (IAM notes, method section 3).
 #include "qk_tile.cuh"
 #include "internal.h"
 
@@ -25,14 +31,15 @@ struct MapsParams {
   int64_t tiles;     // causal tiles per head
   float scale_log2;
   __nv_bfloat16* maps;   // [heads][tiles][64][64]
-  float* norm2;          // [heads]
+  float* norm2;          // [heads] squared norm of the rounded map
+  float* sum1;           // [heads] sum of the rounded map
 };
 
 template <int D>
 __global__ void __launch_bounds__(kTileThreads) maps_kernel(MapsParams p) {
   __shared__ __align__(128) __nv_bfloat16 sK[2 * kTile * D];
   __shared__ __align__(128) __nv_bfloat16 stage[kTile * kTile];
-  __shared__ float red[kTileThreads / 32];
+  __shared__ float red[kTileThreads / 32], red1[kTileThreads / 32];
   const int heads = p.H * p.L_layers;
   const int I = p.nb - 1 - (int)(blockIdx.x / heads);
   const int head = blockIdx.x % heads;
@@ -86,7 +93,7 @@ __global__ void __launch_bounds__(kTileThreads) maps_kernel(MapsParams p) {
 
   // Sweep 2: probabilities as bf16 tiles; squared norm of the rounded values.
   __nv_bfloat16* out = p.maps + ((int64_t)head * p.tiles + (int64_t)I * (I + 1) / 2) * kTile * kTile;
-  float nrm = 0.f;
+  float nrm = 0.f, tot = 0.f;
   load_k_tile<D>(sK0, kb, rs, 0, L, tid);
   cp_async_commit();
   for (int J = 0; J <= I; ++J) {
@@ -105,6 +112,7 @@ __global__ void __launch_bounds__(kTileThreads) maps_kernel(MapsParams p) {
       const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa));
       const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb));
       nrm += fa.x * fa.x + fa.y * fa.y + fb.x * fb.x + fb.y * fb.y;
+      tot += (fa.x + fa.y) + (fb.x + fb.y);
       *reinterpret_cast<uint32_t*>(stage + rA * kTile + ((nt ^ (rA & 7)) << 3) + 2 * t4) = wa;
       *reinterpret_cast<uint32_t*>(stage + rB * kTile + ((nt ^ (rB & 7)) << 3) + 2 * t4) = wb;
     }
@@ -116,10 +124,19 @@ __global__ void __launch_bounds__(kTileThreads) maps_kernel(MapsParams p) {
     }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
-  if (lane == 0) red[warp] = nrm;
+  for (int o = 16; o > 0; o >>= 1) {
+    nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
+    tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  }
+  if (lane == 0) {
+    red[warp] = nrm;
+    red1[warp] = tot;
+  }
   __syncthreads();
-  if (tid == 0) atomicAdd(p.norm2 + head, red[0] + red[1] + red[2] + red[3]);
+  if (tid == 0) {
+    atomicAdd(p.norm2 + head, red[0] + red[1] + red[2] + red[3]);
+    atomicAdd(p.sum1 + head, red1[0] + red1[1] + red1[2] + red1[3]);
+  }
 }
 
 // C_raw[M x N] += A[M x K] . B[N x K]^T over one K split. 128 x 128 output tile, 8 warps of
@@ -219,18 +236,31 @@ __global__ void __launch_bounds__(kGThreads) gram_kernel(GramParams p) {
       }
 }
 
-// One warp per large head: cosine row and argmax (ties: lowest index).
+// One warp per large head: similarity row and argmax (ties: lowest index).
 __global__ void finalize_kernel(const float* __restrict__ craw, const float* __restrict__ n2_large,
-                                const float* __restrict__ n2_small, int M, int N,
-                                float* __restrict__ sim, int32_t* __restrict__ argmax) {
+                                const float* __restrict__ n2_small, const float* __restrict__ s1_large,
+                                const float* __restrict__ s1_small, int M, int N, int metric,
+                                float n_elems, float* __restrict__ sim, int32_t* __restrict__ argmax) {
   const int m = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (m >= M) return;
-  const float nl = sqrtf(n2_large[m]);
+  const float nl2 = n2_large[m], sl = s1_large[m];
+  const float inv_n = 1.f / n_elems;
+  const float var_l = fmaxf(nl2 - sl * sl * inv_n, 0.f);
   float best = -INFINITY;
   int bi = 0x7fffffff;
   for (int s = lane; s < N; s += 32) {
-    const float c = craw[(int64_t)m * N + s] / (nl * sqrtf(n2_small[s]));
+    const float cr = craw[(int64_t)m * N + s];
+    float c;
+    if (metric == IAMAP_SIM_PEARSON) {
+      const float ss = s1_small[s];
+      const float var_s = fmaxf(n2_small[s] - ss * ss * inv_n, 0.f);
+      c = (cr - sl * ss * inv_n) / sqrtf(var_l * var_s);
+    } else if (metric == IAMAP_SIM_EUCLIDEAN) {
+      c = -sqrtf(fmaxf(nl2 + n2_small[s] - 2.f * cr, 0.f));
+    } else {
+      c = cr / (sqrtf(nl2) * sqrtf(n2_small[s]));
+    }
     if (sim) sim[(int64_t)m * N + s] = c;
     if (c > best) {
       best = c;
@@ -249,6 +279,31 @@ __global__ void finalize_kernel(const float* __restrict__ craw, const float* __r
   if (lane == 0) argmax[m] = bi;
 }
 
+// agree = number of i < n with a[i] == b[i] (one CTA).
+__global__ void __launch_bounds__(1024) consistency_kernel(const int32_t* __restrict__ a,
+                                                           const int32_t* __restrict__ b, int n,
+                                                           int32_t* __restrict__ agree) {
+  __shared__ int part[32];
+  int c = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) c += a[i] == b[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += part[w];
+    *agree = t;
+  }
+}
+
+int consistency_impl(const int32_t* a, const int32_t* b, int n, int32_t* agree,
+                     cudaStream_t stream) {
+  consistency_kernel<<<1, 1024, 0, stream>>>(a, b, n, agree);
+  IAMAP_LAUNCH_CHECK("consistency_kernel");
+  return IAMAP_OK;
+}
+
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct HmLayout {
@@ -265,7 +320,7 @@ static HmLayout hm_layout(int L_s, int H_small, int L_l, int H_large, int n_used
   const size_t NS = (size_t)L_s * H_small, NL = (size_t)L_l * H_large;
   l.maps_small = align256(per_head * NS);
   l.maps_large = align256(per_head * NL);
-  l.norms = align256(sizeof(float) * (NS + NL));
+  l.norms = align256(sizeof(float) * 2 * (NS + NL));   // squared norms, then sums
   l.craw = align256(sizeof(float) * NS * NL);
   l.total = l.maps_small + l.maps_large + l.norms + l.craw;
   return l;
@@ -307,6 +362,7 @@ int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream) {
   ps.scale_log2 = kLog2e / sqrtf((float)a.d_small);
   ps.maps = maps_small;
   ps.norm2 = norms;
+  ps.sum1 = norms + NS + NL;
   int rc = a.d_small == 64 ? launch_maps<64>(ps, stream) : launch_maps<128>(ps, stream);
   if (rc) return rc;
   MapsParams pl = ps;
@@ -317,6 +373,7 @@ int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream) {
   pl.scale_log2 = kLog2e / sqrtf((float)a.d_large);
   pl.maps = maps_large;
   pl.norm2 = norms + NS;
+  pl.sum1 = norms + NS + NL + NS;
   rc = a.d_large == 64 ? launch_maps<64>(pl, stream) : launch_maps<128>(pl, stream);
   if (rc) return rc;
 
@@ -340,8 +397,9 @@ int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream) {
                                         (int)gsmem));
   gram_kernel<<<dim3(tm, tn, splits), kGThreads, gsmem, stream>>>(gp);
   IAMAP_LAUNCH_CHECK("gram_kernel");
-  finalize_kernel<<<(NL * 32 + 255) / 256, 256, 0, stream>>>(craw, norms + NS, norms, NL, NS,
-                                                            a.sim, a.argmax);
+  finalize_kernel<<<(NL * 32 + 255) / 256, 256, 0, stream>>>(
+      craw, norms + NS, norms, norms + NS + NL + NS, norms + NS + NL, NL, NS, a.metric,
+      (float)a.n_used * (float)a.n_used, a.sim, a.argmax);
   IAMAP_LAUNCH_CHECK("finalize_kernel");
   return IAMAP_OK;
 }

@@ -63,6 +63,7 @@ struct MappedAvArgs {
   int64_t capacity = 0;
   const float* W = nullptr;
   int H_r = 0;
+  int H_kv = 0;   // value heads; 0 = H_r
   const void* v = nullptr;
   int d_v = 0;
   float* out = nullptr;
@@ -85,6 +86,7 @@ struct PagedArgs {
   const int32_t* ctx_lens = nullptr;
   int max_ctx = 0;
   int batch = 0, H_s = 0, H_r = 0, d_v = 0;
+  int H_kv = 0;   // value heads of the page pool; 0 = H_r
   float* out = nullptr;
   float* partial = nullptr;  // [batch][chunks][H_r][d_v]
   int chunks = 0;            // chunks per sequence
@@ -103,6 +105,7 @@ struct HeadMatchArgs {
   const void* k_large = nullptr;
   int L_l = 0, H_large = 0, d_large = 0;
   int n = 0, n_used = 0;
+  int metric = 0;   // IAMAP_SIM_*
   int32_t* argmax = nullptr;
   float* sim = nullptr;
   void* ws = nullptr;
@@ -110,5 +113,7 @@ struct HeadMatchArgs {
 };
 size_t head_match_ws_bytes(int L_s, int H_small, int L_l, int H_large, int n_used);
 int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream);
+int consistency_impl(const int32_t* a, const int32_t* b, int n, int32_t* agree,
+                     cudaStream_t stream);
 
 }  // namespace iamap

@@ -29,6 +29,7 @@ struct AvParams {
   SeqTables tab;
   int H_s;
   int H_r;
+  int H_kv;     // value heads (H_r / H_kv consecutive receiver heads share one)
   int groups;
   const int32_t* row_ptr;
   const int32_t* col_idx;
@@ -70,7 +71,8 @@ __global__ void __launch_bounds__(kAvThreads, 1) mapped_av_kernel(AvParams p) {
   const int rb = p.tab.rb_start[s] + I;
   const int r0 = grp * kAvGroup;
   const int G = min(kAvGroup, p.H_r - r0);
-  const int64_t vrs = (int64_t)p.H_r * DV;  // V row stride (elements)
+  const int64_t vrs = (int64_t)p.H_kv * DV;  // V row stride (elements)
+  const int kv_grp = p.H_r / p.H_kv;
 
   for (int e = tid; e < kAvGroup * 64; e += kAvThreads) {
     const int r = e / 64, hs = e % 64;
@@ -111,7 +113,8 @@ __global__ void __launch_bounds__(kAvThreads, 1) mapped_av_kernel(AvParams p) {
         const int tok = J * kT + j;
         const bool valid = r < G && tok < L;
         const __nv_bfloat16* src =
-            p.v + (valid ? ((int64_t)(seq0 + tok) * vrs + (int64_t)(r0 + r) * DV + ch * 8) : 0);
+            p.v + (valid ? ((int64_t)(seq0 + tok) * vrs + (int64_t)((r0 + r) / kv_grp) * DV + ch * 8)
+                         : 0);
         const uint32_t dst = smem_u32(sV + r * kT * DV + j * DV + ((ch ^ (j & 7)) << 3));
         cp_async16(dst, src, valid);
       }
@@ -242,6 +245,7 @@ int mapped_av_impl(const MappedAvArgs& a, cudaStream_t stream) {
   p.tab = a.tab;
   p.H_s = a.H_s;
   p.H_r = a.H_r;
+  p.H_kv = a.H_kv > 0 ? a.H_kv : a.H_r;
   p.groups = (a.H_r + kAvGroup - 1) / kAvGroup;
   p.row_ptr = a.row_ptr;
   p.col_idx = a.col_idx;

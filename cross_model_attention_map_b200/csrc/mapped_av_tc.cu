@@ -138,6 +138,7 @@ struct __align__(64) Params {
   float* out;
   unsigned int* status;
   int H_s, H_r, d_v, C, NR, KH, RB, NP;
+  int grp;                 // receiver heads per value head (grouped values; 1 = one each)
   uint32_t off_p, off_w, off_scr, off_recv, off_v, off_wf, off_bar;
 };
 
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         for (int rl = vw; rl < G; rl += kVWarps) {
           tc::mbar_expect_tx(bar_addr(bars, V_FULL + rl), v_stage);
           tc::tma_load_3d_hint(sbase + p.off_v + rl * v_stage, &p.v_map, 0, seq0 + J * 64,
-                               (r0 + rl) * halves, bar_addr(bars, V_FULL + rl), pol);
+                               ((r0 + rl) / p.grp) * halves, bar_addr(bars, V_FULL + rl), pol);
         }
       }
       if (T > 0)
@@ -429,11 +430,23 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
           if (lane == 0) tc::mbar_arrive(bar_addr(bars, D_EMPTY + gs));
           ++gp;
         }
-        // transpose: position = lane, head = register  ->  16-byte runs of one head
+        // transpose: position = lane, head = register  ->  16-byte runs of one head. Lanes 2m and
+        // 2m+1 swap one value per head pair, so that each stores one bf16x2 word: positions
+        // (2m, 2m+1) of the even head (even lane) or of the odd head (odd lane).
+        {
+          const bool odd = lane & 1;
+          uint32_t* scr32 = reinterpret_cast<uint32_t*>(scr);
 #pragma unroll
-        for (int r = 0; r < 32; ++r)
-          if (r < p.NR)
-            reinterpret_cast<__nv_bfloat16*>(scr)[r * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[r]));
+          for (int r = 0; r < 32; r += 2) {
+            if (r < p.NR) {
+              const float mine = __uint_as_float(odd ? v[r + 1] : v[r]);
+              const float send = __uint_as_float(odd ? v[r] : v[r + 1]);
+              const float got = __shfl_xor_sync(0xffffffffu, send, 1);
+              const uint32_t w = odd ? pack_bf16(got, mine) : pack_bf16(mine, got);
+              scr32[(r + (odd ? 1 : 0)) * 16 + (lane >> 1)] = w;
+            }
+          }
+        }
         __syncwarp();
         const int pos0 = 32 * e;                          // this warp's first position in the chunk
         const int arow = 2 * ch + (pos0 >> 6);            // tile row
@@ -546,8 +559,10 @@ int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream) {
     int rc = encode_tmap_2d_bf16(&p.p_maps[i], a.vals, 64, cap * 64, 128, 64, (uint32_t)(8 * (i + 1)));
     if (rc) return rc;
   }
-  int rc = encode_tmap_3d_bf16(&p.v_map, a.v, 64, (uint64_t)a.n, (uint64_t)a.H_r * (a.d_v / 64),
-                               (uint64_t)a.H_r * a.d_v * 2, 128, 64, 64, (uint32_t)(a.d_v / 64));
+  const int H_kv = a.H_kv > 0 ? a.H_kv : a.H_r;
+  p.grp = a.H_r / H_kv;
+  int rc = encode_tmap_3d_bf16(&p.v_map, a.v, 64, (uint64_t)a.n, (uint64_t)H_kv * (a.d_v / 64),
+                               (uint64_t)H_kv * a.d_v * 2, 128, 64, 64, (uint32_t)(a.d_v / 64));
   if (rc) return rc;
   p.cu = a.cu_seqlens;
   p.tab = a.tab;

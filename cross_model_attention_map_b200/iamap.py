@@ -54,7 +54,11 @@ _SIGS = {
                             _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _SZ, _P]),
     "iamap_mapped_av": (_I, [_P, _P, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _I64, _P, _I, _P,
                              _I, _P, _P, _SZ, _P]),
+    "iamap_mapped_av_gqa": (_I, [_P, _P, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _I64, _P, _I, _I,
+                                 _P, _I, _P, _P, _SZ, _P]),
     "iamap_mapped_av_paged_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+    "iamap_mapped_av_paged_gqa": (_I, [_P, _I, _P, _P, _I64, _P, _I, _I, _P, _P, _I, _I, _I, _I,
+                                       _I, _P, _P, _SZ, _P]),
     "iamap_mapped_av_paged": (_I, [_P, _I, _P, _P, _I64, _P, _I, _I, _P, _P, _I, _I, _I, _I,
                                    _P, _P, _SZ, _P]),
     "iamap_mapped_av_paged_noalloc": (_I, [_P, _I, _P, _P, _I64, _P, _I, _I, _P, _P, _I, _I, _I,
@@ -62,6 +66,9 @@ _SIGS = {
     "iamap_head_match_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "iamap_head_match": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ,
                               _P]),
+    "iamap_head_match_metric": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P,
+                                     _P, _SZ, _P]),
+    "iamap_mapping_consistency": (_I, [_P, _P, _I, _P, _P]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -183,6 +190,28 @@ def iamap_mapped_av_paged_workspace_bytes(batch, H_r, d_v, max_ctx, page_size) -
     return _lib.iamap_mapped_av_paged_workspace_bytes(batch, H_r, d_v, max_ctx, page_size)
 
 
+def iamap_mapped_av_gqa(cu_seqlens, cu_seqlens_host, num_seqs, n, B, H_s, row_ptr, col_idx,
+                        headmask, val_off, vals, vals_capacity_tiles, W, H_r, H_kv, v, d_v, out, ws,
+                        stream=None):
+    cp, keep = _host_i32(cu_seqlens_host)
+    _check("iamap_mapped_av_gqa", _lib.iamap_mapped_av_gqa(
+        _ptr(cu_seqlens), cp, num_seqs, n, B, H_s, _ptr(row_ptr), _ptr(col_idx), _ptr(headmask),
+        _ptr(val_off), _ptr(vals), vals_capacity_tiles, _ptr(W), H_r, H_kv, _ptr(v), d_v,
+        _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def iamap_mapped_av_paged_gqa(p_rows, ctx_stride, W, v_pages, num_pages, page_table, max_pages,
+                              page_size, ctx_lens, ctx_lens_host, batch, H_s, H_r, H_kv, d_v, out,
+                              ws, stream=None):
+    cp, keep = _host_i32(ctx_lens_host)
+    _check("iamap_mapped_av_paged_gqa", _lib.iamap_mapped_av_paged_gqa(
+        _ptr(p_rows), ctx_stride, _ptr(W), _ptr(v_pages), num_pages, _ptr(page_table), max_pages,
+        page_size, _ptr(ctx_lens), cp, batch, H_s, H_r, H_kv, d_v, _ptr(out), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
 def iamap_mapped_av_paged(p_rows, ctx_stride, W, v_pages, num_pages, page_table, max_pages,
                           page_size, ctx_lens, ctx_lens_host, batch, H_s, H_r, d_v, out, ws,
                           stream=None):
@@ -208,6 +237,24 @@ def iamap_mapped_av_paged_noalloc(p_rows, ctx_stride, W, v_pages, num_pages, pag
 
 def iamap_head_match_workspace_bytes(L_s, H_small, L_l, H_large, n_used) -> int:
     return _lib.iamap_head_match_workspace_bytes(L_s, H_small, L_l, H_large, n_used)
+
+
+IAMAP_SIM_COSINE, IAMAP_SIM_PEARSON, IAMAP_SIM_EUCLIDEAN = 0, 1, 2
+SIM_METRICS = {"cosine": IAMAP_SIM_COSINE, "pearson": IAMAP_SIM_PEARSON,
+               "euclidean": IAMAP_SIM_EUCLIDEAN}
+
+
+def iamap_head_match_metric(q_small, k_small, L_s, H_small, d_small, q_large, k_large, L_l,
+                            H_large, d_large, n, n_used, metric, argmax, sim, ws, stream=None):
+    _check("iamap_head_match_metric", _lib.iamap_head_match_metric(
+        _ptr(q_small), _ptr(k_small), L_s, H_small, d_small, _ptr(q_large), _ptr(k_large), L_l,
+        H_large, d_large, n, n_used, metric, _ptr(argmax), _ptr(sim), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def iamap_mapping_consistency(a, b, n_heads, agree, stream=None):
+    _check("iamap_mapping_consistency", _lib.iamap_mapping_consistency(
+        _ptr(a), _ptr(b), n_heads, _ptr(agree), _stream(stream)))
 
 
 def iamap_head_match(q_small, k_small, L_s, H_small, d_small, q_large, k_large, L_l, H_large,

@@ -20,7 +20,7 @@ from . import iamap as C
 
 class PrefillLayer:
     def __init__(self, seqlens, H_s, d, H_r, d_v, tau, bias_window=0, bias_value=0.0, B=64,
-                 capacity_tiles=None, device="cuda"):
+                 capacity_tiles=None, device="cuda", H_kv=None):
         self.seqlens = [int(x) for x in seqlens]
         self.num_seqs = len(self.seqlens)
         cu = [0]
@@ -30,6 +30,7 @@ class PrefillLayer:
         self.cu = self.cu_host.to(device)
         self.n = cu[-1]
         self.H_s, self.d, self.H_r, self.d_v, self.B = H_s, d, H_r, d_v, B
+        self.H_kv = H_r if H_kv is None else int(H_kv)   # receiver value heads (grouped if < H_r)
         self.tau, self.bias_window, self.bias_value = float(tau), int(bias_window), float(bias_value)
         self.nrb, self.ncb, self.max_nb = C.iamap_plan(self.cu_host, self.num_seqs, B)
         self.bufs = C.alloc_compress_outputs(self.n, H_s, self.nrb, self.ncb, device)
@@ -49,9 +50,10 @@ class PrefillLayer:
 
     def mapped_av(self, W, v, stream=None):
         b = self.bufs
-        C.iamap_mapped_av(self.cu, self.cu_host, self.num_seqs, self.n, self.B, self.H_s,
-                          b["row_ptr"], b["col_idx"], b["headmask"], b["val_off"], self.vals,
-                          self.capacity, W, self.H_r, v, self.d_v, self.out, self.ws, stream)
+        C.iamap_mapped_av_gqa(self.cu, self.cu_host, self.num_seqs, self.n, self.B, self.H_s,
+                              b["row_ptr"], b["col_idx"], b["headmask"], b["val_off"], self.vals,
+                              self.capacity, W, self.H_r, self.H_kv, v, self.d_v, self.out,
+                              self.ws, stream)
 
     def step(self, q, k, W, v, stream=None):
         self.compress(q, k, stream)
@@ -68,8 +70,9 @@ class DecodeStep:
     """Buffers of one paged decode step on a mapped layer."""
 
     def __init__(self, batch, H_s, H_r, d_v, ctx_lens_host, ctx_stride, max_pages, page_size,
-                 num_pages, device="cuda"):
+                 num_pages, device="cuda", H_kv=None):
         self.batch, self.H_s, self.H_r, self.d_v = batch, H_s, H_r, d_v
+        self.H_kv = H_r if H_kv is None else int(H_kv)
         self.ctx_lens_host = torch.as_tensor(ctx_lens_host, dtype=torch.int32).cpu()
         self.ctx_lens = self.ctx_lens_host.to(device)
         self.ctx_stride, self.max_pages, self.page_size = ctx_stride, max_pages, page_size
@@ -80,10 +83,10 @@ class DecodeStep:
         self.out = torch.empty(batch, H_r, d_v, dtype=torch.float32, device=device)
 
     def run(self, p_rows, W, v_pages, page_table, stream=None):
-        C.iamap_mapped_av_paged(p_rows, self.ctx_stride, W, v_pages, self.num_pages, page_table,
-                                self.max_pages, self.page_size, self.ctx_lens, self.ctx_lens_host,
-                                self.batch, self.H_s, self.H_r, self.d_v, self.out, self.ws,
-                                stream)
+        C.iamap_mapped_av_paged_gqa(p_rows, self.ctx_stride, W, v_pages, self.num_pages,
+                                    page_table, self.max_pages, self.page_size, self.ctx_lens,
+                                    self.ctx_lens_host, self.batch, self.H_s, self.H_r, self.H_kv,
+                                    self.d_v, self.out, self.ws, stream)
         return self.out
 
 
@@ -91,8 +94,9 @@ class HeadMatch:
     """Buffers of one head-matching calibration."""
 
     def __init__(self, L_s, H_small, d_small, L_l, H_large, d_large, n, n_used=None,
-                 want_sim=True, device="cuda"):
+                 want_sim=True, device="cuda", metric="cosine"):
         self.dims = (L_s, H_small, d_small, L_l, H_large, d_large)
+        self.metric = C.SIM_METRICS[metric]
         self.n = n
         self.n_used = n if n_used is None else int(n_used)
         self.ws = C.alloc_workspace(
@@ -103,7 +107,15 @@ class HeadMatch:
 
     def run(self, q_small, k_small, q_large, k_large, stream=None):
         L_s, H_small, d_small, L_l, H_large, d_large = self.dims
-        C.iamap_head_match(q_small, k_small, L_s, H_small, d_small, q_large, k_large, L_l,
-                           H_large, d_large, self.n, self.n_used, self.argmax, self.sim, self.ws,
-                           stream)
+        C.iamap_head_match_metric(q_small, k_small, L_s, H_small, d_small, q_large, k_large,
+                                  L_l, H_large, d_large, self.n, self.n_used, self.metric,
+                                  self.argmax, self.sim, self.ws, stream)
         return self.argmax, self.sim
+
+
+def mapping_consistency(argmax_a, argmax_b, stream=None):
+    """Number of large heads (device int32 tensor of one element) that two head mappings send to
+    the same small head; divide by the head count for the consistency rate."""
+    agree = torch.zeros(1, dtype=torch.int32, device=argmax_a.device)
+    C.iamap_mapping_consistency(argmax_a, argmax_b, argmax_a.numel(), agree, stream)
+    return agree

@@ -78,6 +78,12 @@ extern "C" {
 #define IAMAP_DEV_TIMEOUT    2
 #define IAMAP_DEV_BAD_INDEX  4
 
+/* Similarity of flattened attention maps for head matching (IAM notes, method section 1, which
+ * compares cosine similarity, Minkowski distance and the Pearson correlation). */
+#define IAMAP_SIM_COSINE     0   /* a.b / (|a| |b|) */
+#define IAMAP_SIM_PEARSON    1   /* cosine of a - mean(a) and b - mean(b) over the n_used^2 entries */
+#define IAMAP_SIM_EUCLIDEAN  2   /* -|a - b| (Minkowski distance with p = 2, negated: larger = closer) */
+
 /* Library version, (major << 16) | minor. */
 int iamap_version(void);
 
@@ -163,6 +169,18 @@ int iamap_mapped_av(const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, i
                     float* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * mapped_av with grouped receiver values (grouped-query attention in the receiver): v is bf16
+ * [n, H_kv, d_v] and receiver head r reads value head r / (H_r / H_kv). H_kv must divide H_r
+ * (IAMAP_ERR_INVALID_ARG otherwise); H_kv = H_r is iamap_mapped_av.
+ */
+int iamap_mapped_av_gqa(const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int num_seqs,
+                        int64_t n, int B, int H_s, const int32_t* row_ptr, const int32_t* col_idx,
+                        const uint64_t* headmask, const int64_t* val_off, const void* vals,
+                        int64_t vals_capacity_tiles, const float* W, int H_r, int H_kv,
+                        const void* v, int d_v, float* out, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/*
  * Decode step on a mapped layer: one query row per sequence b.
  *   out[b, r, :] = sum_{j < ctx_lens[b]} (sum_s W[r, s] * p_rows[b, s, j]) * V[b, j, r, :]
  * p_rows  fp32 [batch, H_s, ctx_stride]  the sender's attention rows
@@ -178,6 +196,17 @@ int iamap_mapped_av_paged(const float* p_rows, int ctx_stride, const float* W,
                           int max_pages, int page_size, const int32_t* ctx_lens,
                           const int32_t* ctx_lens_host, int batch, int H_s, int H_r, int d_v,
                           float* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Decode step with grouped receiver values: v_pages bf16 [num_pages, page_size, H_kv, d_v];
+ * receiver head r reads value head r / (H_r / H_kv). H_kv must divide H_r. The workspace is
+ * that of iamap_mapped_av_paged for the same H_r.
+ */
+int iamap_mapped_av_paged_gqa(const float* p_rows, int ctx_stride, const float* W,
+                              const void* v_pages, int64_t num_pages, const int32_t* page_table,
+                              int max_pages, int page_size, const int32_t* ctx_lens,
+                              const int32_t* ctx_lens_host, int batch, int H_s, int H_r, int H_kv,
+                              int d_v, float* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * The paged decode step of iamap_mapped_av_paged for callers that cannot allocate device memory
@@ -217,6 +246,27 @@ int iamap_head_match(const void* q_small, const void* k_small, int L_s, int H_sm
                      const void* q_large, const void* k_large, int L_l, int H_large, int d_large,
                      int n, int n_used, int32_t* argmax, float* sim, void* ws, size_t ws_bytes,
                      void* stream);
+
+/*
+ * Head matching with another similarity: as iamap_head_match, with metric one of IAMAP_SIM_*.
+ * sim then holds that metric (for IAMAP_SIM_EUCLIDEAN the negated distance) and argmax its
+ * largest value per large head. The workspace is the same. An unknown metric returns
+ * IAMAP_ERR_INVALID_ARG.
+ */
+int iamap_head_match_metric(const void* q_small, const void* k_small, int L_s, int H_small,
+                            int d_small, const void* q_large, const void* k_large, int L_l,
+                            int H_large, int d_large, int n, int n_used, int metric,
+                            int32_t* argmax, float* sim, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Mapping consistency (IAM notes, method section 3: the mapping found at prefill holds during
+ * decode). a, b: int32 device arrays of n_heads small-head indices, e.g. the argmax of
+ * iamap_head_match on the prompt and on a longer prefix. *agree (device int32) receives the
+ * number of positions where they are equal; the consistency rate is agree / n_heads.
+ * Asynchronous on stream.
+ */
+int iamap_mapping_consistency(const int32_t* a, const int32_t* b, int n_heads, int32_t* agree,
+                              void* stream);
 
 #ifdef __cplusplus
 }

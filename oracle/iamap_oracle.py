@@ -59,7 +59,7 @@ __all__ = [
     "NEAR_EPS", "CausalLayout", "causal_layout", "head_rows", "scores", "softmax_rows",
     "block_masses", "select_blocks", "RowBlockStats", "rowblock_stats", "CompressResult",
     "compress", "union_bsr", "masked_tile", "mapped_av_rows", "mapped_av", "mapped_av_paged",
-    "attention_map", "head_match", "mapping_consistency",
+    "attention_map", "head_match", "mapping_consistency", "receiver_values",
 ]
 
 
@@ -285,6 +285,16 @@ def masked_tile(st: RowBlockStats, J: int, B: int) -> np.ndarray:
 # Mapped attention output [MapFlow-maps], [MapFlow-C3], [GLIDE II-B]
 # ----------------------------------------------------------------------------------------------
 
+def receiver_values(V: np.ndarray, H_r: int) -> np.ndarray:
+    """The value vectors each receiver head uses: V [tokens, H_kv, d_v] with H_kv dividing H_r;
+    with grouped values (H_kv < H_r) receiver head r reads value head r // (H_r / H_kv), the
+    consecutive-group sharing of grouped-query attention. Returns [tokens, H_r, d_v]."""
+    H_kv = V.shape[1]
+    if H_r % H_kv:
+        raise ValueError("H_kv=%d does not divide H_r=%d" % (H_kv, H_r))
+    return V[:, np.arange(H_r) // (H_r // H_kv)]
+
+
 def mapped_av_rows(wl, s: int, I: int, kept_of, stats_of=None) -> np.ndarray:
     """O rows of one row block: O_r[i] = sum_j (sum_s W[r,s] Pt_s[i,j]) V_r[j], with Pt_s the
     sender head's probabilities restricted to its kept blocks (zero elsewhere).
@@ -306,7 +316,7 @@ def mapped_av_rows(wl, s: int, I: int, kept_of, stats_of=None) -> np.ndarray:
             kmask[J * B:(J + 1) * B] = True
         pt = np.where(kmask[None, :], st.p, 0.0)
         Pr += wl.W[:, h].astype(np.float64)[:, None, None] * pt[None, :, :]
-    V = bf16_bits_to_f64(wl.v[a:b])          # [L, H_r, d_v]
+    V = receiver_values(bf16_bits_to_f64(wl.v[a:b]), wl.H_r)   # [L, H_r, d_v]
     O = np.einsum("rij,jre->ire", Pr, V)
     return O
 
@@ -335,7 +345,7 @@ def mapped_av_paged(dw) -> np.ndarray:
         c = int(dw.ctx_lens[b])
         pr = W @ dw.p_rows[b, :, :c].astype(np.float64)            # [H_r, c]
         pages = dw.page_table[b, (np.arange(c) // ps)]
-        V = bf16_bits_to_f64(dw.v_pages[pages, np.arange(c) % ps])  # [c, H_r, d_v]
+        V = receiver_values(bf16_bits_to_f64(dw.v_pages[pages, np.arange(c) % ps]), dw.H_r)
         O[b] = np.einsum("rj,jre->re", pr, V)
     return O
 

@@ -102,12 +102,13 @@ PREFILL_CONFIGS = {
 
 def make_prefill(seqlens, H_s, d, H_r, d_v, B=64, tau=0.95, std=1.5, sink=True,
                  bias_window=0, bias_value=0.0, seed=0, name="custom",
-                 q_zero=False, v_const=None) -> PrefillWorkload:
+                 q_zero=False, v_const=None, H_kv=None) -> PrefillWorkload:
     """Draw Q, K, V (bf16) and W (fp32) in the order Q, K, V, W.
 
     ``sink`` multiplies the key of token 0 of every sequence by 4 (a power of two, so exact) before
     bf16 rounding. ``q_zero`` zeroes Q (uniform attention rows); ``v_const`` replaces V by that
-    constant. Both are for closed-form checks.
+    constant. Both are for closed-form checks. ``H_kv`` (dividing H_r) draws grouped receiver
+    values: V has H_kv heads.
     """
     seqlens = [int(x) for x in seqlens]
     n = int(sum(seqlens))
@@ -116,7 +117,7 @@ def make_prefill(seqlens, H_s, d, H_r, d_v, B=64, tau=0.95, std=1.5, sink=True,
     rng = np.random.default_rng(seed)
     q = _normal_bits(rng, (n, H_s, d), std)
     k = _normal_bits(rng, (n, H_s, d), std)
-    v = _normal_bits(rng, (n, H_r, d_v), std)
+    v = _normal_bits(rng, (n, H_r if H_kv is None else int(H_kv), d_v), std)
     W = rng.standard_normal((H_r, H_s), dtype=np.float32) * np.float32(math.sqrt(1.0 / H_s))
     if sink:
         for s in range(len(seqlens)):
@@ -207,12 +208,13 @@ class DecodeWorkload:
 
 
 def make_decode(batch=4, ctx=8704, H_s=14, H_r=64, d_v=128, page_size=16, sink_weight=64.0,
-                ctx_lens=None, seed=0) -> DecodeWorkload:
+                ctx_lens=None, seed=0, H_kv=None) -> DecodeWorkload:
     """Draw order: sender rows, one-hot assignment, V pages, page-table permutation.
 
     The sender's attention rows are drawn from a Dirichlet distribution (normalised Gamma draws)
     with a heavier concentration at position 0, a stand-in for a causal softmax row with a sink.
-    Unused tail positions (ctx_len < max) are zero.
+    Unused tail positions (ctx_len < max) are zero. ``H_kv`` (dividing H_r) gives the page
+    pool that many value heads.
     """
     if ctx_lens is None:
         ctx_lens = [ctx] * batch
@@ -231,7 +233,8 @@ def make_decode(batch=4, ctx=8704, H_s=14, H_r=64, d_v=128, page_size=16, sink_w
     W = np.zeros((H_r, H_s), dtype=np.float32)
     W[np.arange(H_r), assign] = 1.0
     num_pages = batch * max_pages
-    v = rng.standard_normal((num_pages, page_size, H_r, d_v), dtype=np.float32)
+    v = rng.standard_normal((num_pages, page_size, H_r if H_kv is None else int(H_kv), d_v),
+                            dtype=np.float32)
     perm = rng.permutation(num_pages).astype(np.int32)
     page_table = perm.reshape(batch, max_pages)
     return DecodeWorkload(batch=batch, ctx_lens=ctx_lens, H_s=H_s, H_r=H_r, d_v=d_v,

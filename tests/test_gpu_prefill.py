@@ -30,7 +30,7 @@ def C():
 def _run(wl, capacity=None):
     from cross_model_attention_map_b200.runner import PrefillLayer
     layer = PrefillLayer(wl.seqlens, wl.H_s, wl.d, wl.H_r, wl.d_v, wl.tau, wl.bias_window,
-                         wl.bias_value, capacity_tiles=capacity)
+                         wl.bias_value, capacity_tiles=capacity, H_kv=wl.v.shape[1])
     q, k, v, W = upload_prefill(wl)
     layer.step(q, k, W, v)
     torch.cuda.synchronize()
@@ -100,6 +100,18 @@ def test_tiny_config_full_parity(C):
 def test_varlen_parity(C, seqlens, H_s, H_r, d, tau, bias):
     wl = make_prefill(seqlens, H_s=H_s, d=d, H_r=H_r, d_v=d, B=64, tau=tau, std=1.5, sink=True,
                       bias_window=bias[0], bias_value=bias[1], seed=21)
+    _full_parity(C, wl)
+
+
+@pytest.mark.parametrize("seqlens,H_s,H_r,H_kv,d", [
+    ([300, 90], 6, 8, 2, 64),      # tensor-core cluster kernel, 4 receivers per value head
+    ([200], 5, 12, 3, 128),        # tensor-core, groups across CTA boundaries
+    ([260, 40], 4, 40, 8, 64),     # H_r > 32: the CUDA-core kernel
+])
+def test_grouped_values_parity(C, seqlens, H_s, H_r, H_kv, d):
+    """Grouped receiver values (receiver head r reads value head r / (H_r / H_kv))."""
+    wl = make_prefill(seqlens, H_s=H_s, d=d, H_r=H_r, d_v=d, B=64, tau=0.9, std=1.5, sink=True,
+                      seed=43, H_kv=H_kv)
     _full_parity(C, wl)
 
 

@@ -421,3 +421,20 @@ def test_head_match_planted_full_size():
     np.testing.assert_array_equal(arg, hm.planted)
     top2 = np.sort(C, axis=1)[:, -2:]
     assert (top2[:, 1] - top2[:, 0]).min() > 0.05
+
+
+def test_grouped_values_equal_repeated_heads():
+    """Grouped receiver values (H_kv < H_r): the output equals that of a workload whose V holds
+    every value head repeated H_r / H_kv times in consecutive receiver heads (prefill and decode)."""
+    import dataclasses
+    wl = make_prefill([150, 70], H_s=4, d=16, H_r=6, d_v=8, B=16, tau=0.9, seed=41, H_kv=2)
+    lay = O.causal_layout(wl.seqlens, wl.B)
+    kept = np.ones((wl.H_s, lay.num_causal_blocks), dtype=bool)
+    rep = dataclasses.replace(wl, v=np.repeat(wl.v, 3, axis=1))
+    assert rep.v.shape[1] == 6
+    np.testing.assert_array_equal(O.mapped_av(wl, kept), O.mapped_av(rep, kept))
+    dw = make_decode(batch=2, ctx=70, H_s=3, H_r=8, d_v=8, page_size=16, seed=42, H_kv=2)
+    drep = dataclasses.replace(dw, v_pages=np.repeat(dw.v_pages, 4, axis=2))
+    np.testing.assert_array_equal(O.mapped_av_paged(dw), O.mapped_av_paged(drep))
+    with pytest.raises(ValueError):
+        O.receiver_values(np.zeros((3, 4, 2)), 6)
