@@ -8,8 +8,9 @@
 //    writes them as bf16 64 x 64 tiles in causal-block order, zeros above the diagonal and past
 //    n_used. The flattened map of a head is its run of tiles. The squared norm of the bf16 map is
 //    accumulated alongside.
-// 2. gram_kernel: C_raw = A_large . A_small^T over the flattened maps (split-K, mma.sync,
-//    fp32 accumulate, atomic fp32 reduction of the K splits).
+// 2. gram_tc_kernel: C_raw = A_large . A_small^T over the flattened maps on the tcgen05 tensor
+//    cores (split-K; operands by TMA with 128-byte swizzle, fp32 accumulator in TMEM, atomic fp32
+//    reduction of the K splits).
 // 3. finalize_kernel: the similarity of every (large, small) pair from C_raw and each map's sum and
 //    squared norm, and the argmax per large head (lowest small-head index on ties). The method
 //    section of the IAM notes compares cosine similarity, Minkowski distance and the Pearson
@@ -18,7 +19,10 @@
 //    |a - b|^2 = |a|^2 + |b|^2 - 2 C, reported negated so that larger is more similar.
 // 4. consistency_kernel: how many large heads two mappings (e.g. prefill and a later prefix)
 //    send to the same small head (IAM notes, method section 3).
+#include <algorithm>
+
 #include "qk_tile.cuh"
+#include "tc_utils.cuh"
 #include "internal.h"
 
 namespace iamap {
@@ -139,101 +143,116 @@ __global__ void __launch_bounds__(kTileThreads) maps_kernel(MapsParams p) {
   }
 }
 
-// C_raw[M x N] += A[M x K] . B[N x K]^T over one K split. 128 x 128 output tile, 8 warps of
-// 64 x 32, K staged 64 at a time through a 3-stage cp.async ring with a 16-byte XOR swizzle.
-constexpr int kGBM = 128, kGBN = 128, kGBK = 64, kGStages = 3, kGThreads = 256;
+// ------------------------------------------------------------------------------------------------
+// Gram on tcgen05: CTA (M tile of 128 large heads, N tile of BN small heads, K split). Warp 0
+// loads A, warp 1 loads B (one 64-element K step per stage, 5 stages), lane 0 of warp 2 issues
+// 4 MMAs (128 x BN x 16) per stage and frees the stage with a commit; warps 2-5 then read the
+// accumulator (TMEM lane = large head, column = small head) and add it into C.
+// ------------------------------------------------------------------------------------------------
+constexpr int kGtStages = 5, kGtThreads = 192;
 
-struct GramParams {
-  const __nv_bfloat16* A;
-  const __nv_bfloat16* B;
-  int M, N;
-  int64_t K;
-  int64_t k_per_split;
+struct GramTcParams {
+  CUtensorMap a_map;   // maps_large viewed [M][K] bf16, box {64, 128}
+  CUtensorMap b_map;   // maps_small viewed [N][K] bf16, box {64, BN}
+  int M, N, BN;
+  int64_t K, k_per_split;
   float* C;
+  unsigned int* status;
 };
 
-__global__ void __launch_bounds__(kGThreads) gram_kernel(GramParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  __nv_bfloat16* sA = reinterpret_cast<__nv_bfloat16*>(smem);
-  __nv_bfloat16* sB = sA + kGStages * kGBM * kGBK;
+__global__ void __launch_bounds__(kGtThreads, 1) gram_tc_kernel(const __grid_constant__ GramTcParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t a_stage = 128u * 128u, b_stage = (uint32_t)p.BN * 128u;
+  const uint32_t stage = a_stage + b_stage;
+  uint64_t* bar_mem = reinterpret_cast<uint64_t*>(smem + kGtStages * stage);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bar_mem + 2 * kGtStages + 1);   // [0] tmem [1] abort
+  const uint32_t bars = smem_u32(bar_mem);
+  auto FULL = [&](int i) { return bars + 8u * (uint32_t)i; };
+  auto EMPTY = [&](int i) { return bars + 8u * (uint32_t)(kGtStages + i); };
+  const uint32_t DONE = bars + 8u * (uint32_t)(2 * kGtStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = blockIdx.x * kGBM, n0 = blockIdx.y * kGBN;
+  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * p.BN;
   const int64_t k0 = (int64_t)blockIdx.z * p.k_per_split;
   const int64_t k1 = min(p.K, k0 + p.k_per_split);
-  const int nsteps = (int)((k1 - k0 + kGBK - 1) / kGBK);
-  const int wm = (warp >> 2) * 64, wn = (warp & 3) * 32;
+  const int nsteps = (int)((k1 - k0) / 64);   // K and the split are multiples of 64
 
-  auto load_stage = [&](int step, int buf) {
-    const int64_t kk = k0 + (int64_t)step * kGBK;
-    for (int c = tid; c < kGBM * 8; c += kGThreads) {
-      const int r = c >> 3, ch = c & 7;
-      const bool va = (m0 + r) < p.M && kk + ch * 8 < k1;
-      const __nv_bfloat16* src = p.A + (va ? ((int64_t)(m0 + r) * p.K + kk + ch * 8) : 0);
-      cp_async16(smem_u32(sA + (buf * kGBM + r) * kGBK + ((ch ^ (r & 7)) << 3)), src, va);
-      const bool vb = (n0 + r) < p.N && kk + ch * 8 < k1;
-      const __nv_bfloat16* srb = p.B + (vb ? ((int64_t)(n0 + r) * p.K + kk + ch * 8) : 0);
-      cp_async16(smem_u32(sB + (buf * kGBN + r) * kGBK + ((ch ^ (r & 7)) << 3)), srb, vb);
+  if (tid == 0) {
+    for (int i = 0; i < kGtStages; ++i) {
+      tc::mbar_init(FULL(i), 2);    // one expect_tx arrival from each producer
+      tc::mbar_init(EMPTY(i), 1);
     }
-  };
-
-  float acc[4][4][4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[a][b][e] = 0.f;
-
-  for (int s = 0; s < kGStages - 1; ++s) {
-    if (s < nsteps) load_stage(s, s);
-    cp_async_commit();
+    tc::mbar_init(DONE, 1);
+    misc[1] = 0;
+    tc::fence_barrier_init();
   }
-  const int mq = lane >> 3, rr = lane & 7;
-  for (int step = 0; step < nsteps; ++step) {
-    cp_async_wait<kGStages - 2>();
-    __syncthreads();
-    const int nxt = step + kGStages - 1;
-    if (nxt < nsteps) load_stage(nxt, nxt % kGStages);
-    cp_async_commit();
-    const int buf = step % kGStages;
-    const __nv_bfloat16* A = sA + buf * kGBM * kGBK;
-    const __nv_bfloat16* B = sB + buf * kGBN * kGBK;
-#pragma unroll
-    for (int ks = 0; ks < kGBK / 16; ++ks) {
-      uint32_t af[4][4];
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        const int row = wm + mt * 16 + (mq & 1) * 8 + rr;
-        const int ch = ks * 2 + (mq >> 1);
-        ldmatrix_x4(smem_u32(A + row * kGBK + ((ch ^ (row & 7)) << 3)), af[mt][0], af[mt][1],
-                    af[mt][2], af[mt][3]);
+  if (warp == 2) tc::tmem_alloc(smem_u32(misc), 256);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp < 2) {
+    if (lane == 0) {
+      const CUtensorMap* map = warp == 0 ? &p.a_map : &p.b_map;
+      const uint32_t off = warp == 0 ? 0u : a_stage;
+      const uint32_t bytes = warp == 0 ? a_stage : b_stage;
+      const int y = warp == 0 ? m0 : n0;
+      tc::prefetch_tmap(map);
+      for (int st = 0; st < nsteps; ++st) {
+        const int b = st % kGtStages;
+        if (st >= kGtStages)
+          tc::wait_bar(EMPTY(b), ((st / kGtStages) - 1) & 1, abort_flag, p.status);
+        tc::mbar_expect_tx(FULL(b), bytes);
+        tc::tma_load_2d(sbase + b * stage + off, map, (int)(k0 + (int64_t)st * 64), y, FULL(b));
       }
-#pragma unroll
-      for (int nt2 = 0; nt2 < 2; ++nt2) {
-        const int row = wn + nt2 * 16 + (mq >> 1) * 8 + rr;
-        const int ch = ks * 2 + (mq & 1);
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4(smem_u32(B + row * kGBK + ((ch ^ (row & 7)) << 3)), b0, b1, b2, b3);
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
-          mma_bf16_16816(acc[mt][2 * nt2], af[mt], b0, b1);
-          mma_bf16_16816(acc[mt][2 * nt2 + 1], af[mt], b2, b3);
-        }
-      }
+      for (int st = max(0, nsteps - kGtStages); st < nsteps; ++st)
+        tc::drain_bar(FULL(st % kGtStages), (st / kGtStages) & 1);
     }
-  }
-  cp_async_wait<0>();
-  const int g = lane >> 2, t4 = lane & 3;
+  } else {
+    if (warp == 2 && lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(128, p.BN, 0, 0);
+      for (int st = 0; st < nsteps; ++st) {
+        const int b = st % kGtStages;
+        tc::wait_bar(FULL(b), (st / kGtStages) & 1, abort_flag, p.status);
+        tc::tc_fence_after();
+        const uint32_t sa = sbase + b * stage, sb = sa + a_stage;
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int m = m0 + wm + mt * 16 + g + (e >= 2 ? 8 : 0);
-        const int nn = n0 + wn + nt * 8 + 2 * t4 + (e & 1);
-        if (m < p.M && nn < p.N) atomicAdd(p.C + (int64_t)m * p.N + nn, acc[mt][nt][e]);
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_bf16(tmem, tc::sdesc_sw128(sa + kk * 32u, 16u, 1024u),
+                       tc::sdesc_sw128(sb + kk * 32u, 16u, 1024u), idesc,
+                       (st > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_commit(EMPTY(b));
       }
+      tc::mma_commit(DONE);
+    }
+    __syncwarp();
+    // accumulator readout: warp w reads TMEM lane quarter w % 4
+    tc::wait_bar(DONE, 0, abort_flag, p.status);
+    tc::tc_fence_after();
+    const int q = warp & 3;
+    const int m = m0 + 32 * q + lane;
+    const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
+    for (int c0 = 0; c0 < p.BN; c0 += 16) {
+      uint32_t v[16];
+      IAMAP_TMEM_LD16(t_lane + (uint32_t)c0, v);
+      tc::tmem_ld_wait();
+      if (nsteps > 0 && m < p.M)
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if (n0 + c0 + e < p.N) atomicAdd(p.C + (int64_t)m * p.N + n0 + c0 + e, __uint_as_float(v[e]));
+    }
+    if (warp == 2 && lane == 0) tc::drain_bar(DONE, 0);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 256);
+  }
 }
 
 // One warp per large head: similarity row and argmax (ties: lowest index).
@@ -377,26 +396,36 @@ int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream) {
   rc = a.d_large == 64 ? launch_maps<64>(pl, stream) : launch_maps<128>(pl, stream);
   if (rc) return rc;
 
-  GramParams gp{};
-  gp.A = maps_large;
-  gp.B = maps_small;
-  gp.M = NL;
-  gp.N = NS;
-  gp.K = l.tiles * kTile * kTile;
-  const int tm = (NL + kGBM - 1) / kGBM, tn = (NS + kGBN - 1) / kGBN;
-  DeviceContext* ctx = device_context();
-  const int sms = ctx ? ctx->num_sms : 148;
-  int splits = (2 * sms + tm * tn - 1) / (tm * tn);
-  int64_t kps = (gp.K + splits - 1) / splits;
-  kps = (kps + kGBK - 1) / kGBK * kGBK;
-  splits = (int)((gp.K + kps - 1) / kps);
-  gp.k_per_split = kps;
-  gp.C = craw;
-  const size_t gsmem = (size_t)kGStages * (kGBM + kGBN) * kGBK * 2;
-  IAMAP_CUDA_CHECK(cudaFuncSetAttribute(gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)gsmem));
-  gram_kernel<<<dim3(tm, tn, splits), kGThreads, gsmem, stream>>>(gp);
-  IAMAP_LAUNCH_CHECK("gram_kernel");
+  {
+    GramTcParams gp{};
+    const int64_t K = l.tiles * kTile * kTile;
+    const int ntn = (NS + 255) / 256;                       // N tiles of at most 256 small heads
+    gp.BN = ((NS + ntn - 1) / ntn + 15) / 16 * 16;
+    gp.M = NL;
+    gp.N = NS;
+    gp.K = K;
+    gp.C = craw;
+    gp.status = a.status;
+    int rc2 = encode_tmap_2d_bf16(&gp.a_map, maps_large, (uint64_t)K, (uint64_t)NL,
+                                  (uint64_t)K * 2, 64, 128);
+    if (!rc2) rc2 = encode_tmap_2d_bf16(&gp.b_map, maps_small, (uint64_t)K, (uint64_t)NS,
+                                        (uint64_t)K * 2, 64, (uint32_t)gp.BN);
+    if (rc2) return rc2;
+    const int tm = (NL + 127) / 128, tn = (NS + gp.BN - 1) / gp.BN;
+    DeviceContext* ctx = device_context();
+    const int sms = ctx ? ctx->num_sms : 148;
+    int splits = std::max(1, sms / (tm * tn));
+    int64_t kps = (K + splits - 1) / splits;
+    kps = (kps + 63) / 64 * 64;
+    splits = (int)((K + kps - 1) / kps);
+    gp.k_per_split = kps;
+    const size_t gsmem = 1024 + (size_t)kGtStages * (128 * 128 + (size_t)gp.BN * 128) +
+                         8 * (2 * kGtStages + 1) + 16;
+    IAMAP_CUDA_CHECK(cudaFuncSetAttribute(gram_tc_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem));
+    gram_tc_kernel<<<dim3(tm, tn, splits), kGtThreads, gsmem, stream>>>(gp);
+    IAMAP_LAUNCH_CHECK("gram_tc_kernel");
+  }
   finalize_kernel<<<(NL * 32 + 255) / 256, 256, 0, stream>>>(
       craw, norms + NS, norms, norms + NS + NL + NS, norms + NS + NL, NL, NS, a.metric,
       (float)a.n_used * (float)a.n_used, a.sim, a.argmax);
