@@ -30,7 +30,8 @@ namespace iamap {
 namespace tccomp {
 
 constexpr int kRows = 128;         // query rows per CTA (row blocks 2P, 2P + 1)
-constexpr int kThreads = 320;      // warps 0-7 softmax, 8 TMA, 9 MMA
+constexpr int kThreads = 320;      // extract: warps 0-7 writers, 8 TMA, 9 MMA
+constexpr int kSThreads = 352;     // stats: warps 0-7 softmax, 8 and 10 TMA, 9 MMA
 constexpr int kSoft = 256;         // softmax threads
 constexpr int kSStages = 4;        // stats: key-tile ring (128 keys per tile)
 constexpr int kXStages = 2;        // extract: key-tile ring (64 keys per tile)
@@ -49,6 +50,7 @@ struct StatsParams {
   CUtensorMap q_map;   // {64, n, H_s * D / 64} bf16, box {64, 128, 1}
   CUtensorMap k_map;   // same geometry
   const int32_t* cu;
+  const int32_t* tok0;   // first q/k token of each sequence; null: cu (packed sequences)
   SeqTables tab;
   int64_t n, ncb;
   int H_s;
@@ -57,7 +59,7 @@ struct StatsParams {
   float bias_log2;
   float tau;
   float* lse;
-  float* mass;
+  float* mass;           // null: row statistics only (no masses, no choice)
   unsigned long long* headmask_dense;
   unsigned int* status;
 };
@@ -66,6 +68,7 @@ struct ExtractParams {
   CUtensorMap q_map;   // box {64, 128, 1}
   CUtensorMap k_map;   // box {64, 64, 1}
   const int32_t* cu;
+  const int32_t* tok0;   // as in StatsParams
   SeqTables tab;
   int64_t n;
   int H_s;
@@ -80,6 +83,13 @@ struct ExtractParams {
   __nv_bfloat16* vals;
   int64_t capacity;
   unsigned int* status;
+  // dense mode (head_match maps): every causal tile of every head, head-major, row-major tiles
+  // (tile I(I+1)/2 + J of head (s * H_s + h) at index (s * H_s + h) * dense_tiles + ...), with the
+  // sum and the squared norm of each head's rounded map added into sum1 / norm2
+  int dense;
+  int64_t dense_tiles;
+  float* norm2;
+  float* sum1;
 };
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t bars, int i) { return bars + 8u * (uint32_t)i; }
@@ -184,7 +194,7 @@ __device__ __forceinline__ float block_log2sum(uint32_t (&v)[64], int i, int j0,
 // ------------------------------------------------------------------------------------------------
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_constant__ StatsParams p) {
+__global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_constant__ StatsParams p) {
   constexpr int NPAN = D / 64;
   constexpr uint32_t kQBytes = NPAN * kPanel128;
   constexpr uint32_t kKStage = NPAN * kPanel128;
@@ -210,14 +220,17 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
   const int h = blockIdx.x - pair * p.H_s;
   const int2 it = p.tab.pairs[pair];
   const int s = it.x, I0 = it.y, P = I0 >> 1;
-  const int seq0 = p.cu[s];
-  const int L = p.cu[s + 1] - seq0;
+  const int row0 = p.cu[s];                 // packed row index of the sequence's token 0
+  const int seq0 = p.tok0 ? p.tok0[s] : row0;   // its q/k token
+  const int L = p.cu[s + 1] - row0;
   const int nb = p.tab.nb[s];
   const int nT = P + 1;                     // key tiles of 128
 
   if (tid == 0) {
     for (int i = 0; i < NUM_BARS; ++i)
-      tc::mbar_init(bar_addr(bars, i), (i >= S_EMPTY && i < S_EMPTY + 2) ? 8u : 1u);
+      tc::mbar_init(bar_addr(bars, i), (i >= S_EMPTY && i < S_EMPTY + 2) ? 8u
+                                       : (i >= K_FULL && i < K_FULL + kSStages) ? (uint32_t)NPAN
+                                                                                : 1u);
     misc[1] = 0;
     tc::fence_barrier_init();
   }
@@ -227,29 +240,32 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
   tc::tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  if (warp == 8) {
+  if (warp == 8 || warp == 10) {
     // ------------------------------ TMA: Q once, then the key tiles ------------------------------
-    if (lane == 0) {
-      tc::prefetch_tmap(&p.q_map);
-      tc::prefetch_tmap(&p.k_map);
-      tc::mbar_expect_tx(bar_addr(bars, Q_FULL), kQBytes);
+    // One thread issues a 16 KB box only every ~0.3 us, so the two 64-dim panels of each key tile
+    // come from two warps (warp 8: panel 0 and Q, warp 10: panel 1), each arriving on K_FULL.
+    const int pan = warp == 8 ? 0 : 1;
+    if (lane == 0 && pan < NPAN) {
+      if (pan == 0) {
+        tc::prefetch_tmap(&p.q_map);
+        tc::mbar_expect_tx(bar_addr(bars, Q_FULL), kQBytes);
 #pragma unroll
-      for (int pan = 0; pan < NPAN; ++pan)
-        tc::tma_load_3d(sQ + pan * kPanel128, &p.q_map, 0, seq0 + kRows * P, h * NPAN + pan,
-                        bar_addr(bars, Q_FULL));
+        for (int qp = 0; qp < NPAN; ++qp)
+          tc::tma_load_3d(sQ + qp * kPanel128, &p.q_map, 0, seq0 + kRows * P, h * NPAN + qp,
+                          bar_addr(bars, Q_FULL));
+      }
+      tc::prefetch_tmap(&p.k_map);
       for (int T = 0; T < nT; ++T) {
         const int st = T % kSStages;
         if (T >= kSStages)
           tc::wait_bar(bar_addr(bars, K_EMPTY + st), ((T / kSStages) - 1) & 1, abort_flag, p.status);
-        tc::mbar_expect_tx(bar_addr(bars, K_FULL + st), kKStage);
-#pragma unroll
-        for (int pan = 0; pan < NPAN; ++pan)
-          tc::tma_load_3d(sK + st * kKStage + pan * kPanel128, &p.k_map, 0, seq0 + 128 * T,
-                          h * NPAN + pan, bar_addr(bars, K_FULL + st));
+        tc::mbar_expect_tx(bar_addr(bars, K_FULL + st), kPanel128);
+        tc::tma_load_3d(sK + st * kKStage + pan * kPanel128, &p.k_map, 0, seq0 + 128 * T,
+                        h * NPAN + pan, bar_addr(bars, K_FULL + st));
       }
       for (int T = max(0, nT - kSStages); T < nT; ++T)
         tc::drain_bar(bar_addr(bars, K_FULL + T % kSStages), (T / kSStages) & 1);
-      tc::drain_bar(bar_addr(bars, Q_FULL), 0);
+      if (pan == 0) tc::drain_bar(bar_addr(bars, Q_FULL), 0);
     }
   } else if (warp == 9) {
     // ------------------------------ MMA: S_b = Q K_T^T (128 x 128, fp32 in TMEM) ----------------
@@ -344,9 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
       float lse2 = -INFINITY;
       if (m > -INFINITY) lse2 = m + lg2(ml_l[r] * ex2(m0 - m) + ml_l[kRows + r] * ex2(m1 - m));
       lse_s[r] = lse2;
-      if (valid) p.lse[(int64_t)h * p.n + seq0 + i] = lse2 * kLn2;
+      if (valid) p.lse[(int64_t)h * p.n + row0 + i] = lse2 * kLn2;
     }
     tc::named_bar(1, kSoft);
+    if (p.mass != nullptr) {
 
     // ---- block masses: sum over the valid rows of 2^(c_iJ - lse_i) ----
     const int nJ = min(2 * P + 2, nb);
@@ -411,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
         }
       }
     }
+    }   // masses
   }
 
   tc::tc_fence_before();
@@ -448,8 +466,9 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
   const int h = blockIdx.x - pair * p.H_s;
   const int2 it = p.tab.pairs[pair];
   const int s = it.x, I0 = it.y, P = I0 >> 1;
-  const int seq0 = p.cu[s];
-  const int L = p.cu[s + 1] - seq0;
+  const int row0 = p.cu[s];
+  const int seq0 = p.tok0 ? p.tok0[s] : row0;
+  const int L = p.cu[s + 1] - row0;
   const int nb = p.tab.nb[s];
   const int nJ = min(2 * P + 2, nb);
 
@@ -463,7 +482,15 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
   if (warp == 9) tc::tmem_alloc(smem_u32(misc), 256);
   __syncthreads();
   // this head's stored blocks in row blocks I0 and I1, by column block
-  if (warp < 2 && I0 + warp < nb) {
+  if (p.dense) {
+    for (int idx = tid; idx < 2 * kMaxNb; idx += kThreads) {
+      const int k = idx / kMaxNb, J = idx - k * kMaxNb, I = I0 + k;
+      if (I < nb && J <= I) {
+        base_s[idx] = ((int64_t)s * p.H_s + h) * p.dense_tiles + (int64_t)I * (I + 1) / 2 + J;
+        rk_s[idx] = 1 << 8;
+      }
+    }
+  } else if (warp < 2 && I0 + warp < nb) {
     const int rb = p.tab.rb_start[s] + I0 + warp;
     const int u0 = p.row_ptr[rb], u1 = p.row_ptr[rb + 1];
     const unsigned long long below = (1ull << h) - 1ull;
@@ -550,9 +577,10 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
     const int il = r & 63;                        // row within the tile
     const uint32_t t_lane = (uint32_t)(32 * qd) << 16;
     const float sc = p.scale_log2;
-    const float lse2 = valid ? p.lse[(int64_t)h * p.n + seq0 + i] * kLog2e : 0.f;
+    const float lse2 = valid ? p.lse[(int64_t)h * p.n + row0 + i] * kLog2e : 0.f;
     unsigned char* stg = stage_all + warp * 4096;
     bool cap_flag = false;
+    float acc1 = 0.f, acc2 = 0.f;   // dense mode: sum and squared norm of this row's rounded values
     for (int t = G; t < nU; t += 2) {
       const int b = t & (kXBufs - 1);
       tc::wait_bar(bar_addr(bars, XS_FULL + b), (t >> 2) & 1, abort_flag, p.status);
@@ -595,6 +623,14 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
               pk[e >> 1] = pack_bf16(a[0], a[1]);
             }
           }
+          if (p.norm2) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
+              acc1 += f.x + f.y;
+              acc2 = fmaf(f.x, f.x, fmaf(f.y, f.y, acc2));
+            }
+          }
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const int cc = 4 * half + c;
@@ -625,6 +661,17 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
       __syncwarp();
     }
     if (cap_flag && lane == 0) raise_status(p.status, IAMAP_DEV_CAPACITY);
+    if (p.norm2) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+        acc2 += __shfl_xor_sync(0xffffffffu, acc2, o);
+      }
+      if (lane == 0) {
+        atomicAdd(p.sum1 + (int64_t)s * p.H_s + h, acc1);
+        atomicAdd(p.norm2 + (int64_t)s * p.H_s + h, acc2);
+      }
+    }
   }
 
   tc::tc_fence_before();
@@ -661,10 +708,12 @@ static int encode_qk_map(CUtensorMap* map, const void* base, int64_t n, int H_s,
 int compress_stats_tc_launch(const CompressArgs& a, cudaStream_t stream) {
   using namespace tccomp;
   StatsParams p{};
-  int rc = encode_qk_map(&p.q_map, a.q, a.n, a.H_s, a.d, 128);
-  if (!rc) rc = encode_qk_map(&p.k_map, a.k, a.n, a.H_s, a.d, 128);
+  const int64_t n_tok = a.n_tok > 0 ? a.n_tok : a.n;
+  int rc = encode_qk_map(&p.q_map, a.q, n_tok, a.H_s, a.d, 128);
+  if (!rc) rc = encode_qk_map(&p.k_map, a.k, n_tok, a.H_s, a.d, 128);
   if (rc) return rc;
   p.cu = a.cu_seqlens;
+  p.tok0 = a.tok0;
   p.tab = a.tab;
   p.n = a.n;
   p.ncb = a.plan.num_causal_blocks;
@@ -683,7 +732,7 @@ int compress_stats_tc_launch(const CompressArgs& a, cudaStream_t stream) {
   IAMAP_CUDA_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const int64_t grid = a.plan.num_pairs * a.H_s;
   if (grid > 0) {
-    kern<<<(unsigned)grid, kThreads, smem, stream>>>(p);
+    kern<<<(unsigned)grid, kSThreads, smem, stream>>>(p);
     IAMAP_LAUNCH_CHECK("compress stats (tcgen05)");
   }
   return IAMAP_OK;
@@ -692,10 +741,16 @@ int compress_stats_tc_launch(const CompressArgs& a, cudaStream_t stream) {
 int compress_extract_tc_launch(const CompressArgs& a, cudaStream_t stream) {
   using namespace tccomp;
   ExtractParams p{};
-  int rc = encode_qk_map(&p.q_map, a.q, a.n, a.H_s, a.d, 128);
-  if (!rc) rc = encode_qk_map(&p.k_map, a.k, a.n, a.H_s, a.d, 64);
+  const int64_t n_tok = a.n_tok > 0 ? a.n_tok : a.n;
+  int rc = encode_qk_map(&p.q_map, a.q, n_tok, a.H_s, a.d, 128);
+  if (!rc) rc = encode_qk_map(&p.k_map, a.k, n_tok, a.H_s, a.d, 64);
   if (rc) return rc;
   p.cu = a.cu_seqlens;
+  p.tok0 = a.tok0;
+  p.dense = a.dense;
+  p.dense_tiles = a.dense_tiles;
+  p.norm2 = a.norm2;
+  p.sum1 = a.sum1;
   p.tab = a.tab;
   p.n = a.n;
   p.H_s = a.H_s;

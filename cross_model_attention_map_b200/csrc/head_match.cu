@@ -20,6 +20,7 @@
 // 4. consistency_kernel: how many large heads two mappings (e.g. prefill and a later prefix)
 //    send to the same small head (IAM notes, method section 3).
 #include <algorithm>
+#include <vector>
 
 #include "qk_tile.cuh"
 #include "tc_utils.cuh"
@@ -329,6 +330,8 @@ struct HmLayout {
   int nb;
   int64_t tiles;
   size_t maps_small, maps_large, norms, craw, total;
+  // tensor-core maps: per model, row log-sum-exp, scheduling tables, cu and token offsets
+  size_t lse_small, lse_large, tab_small, tab_large, seq_small, seq_large;
 };
 
 static HmLayout hm_layout(int L_s, int H_small, int L_l, int H_large, int n_used) {
@@ -341,7 +344,14 @@ static HmLayout hm_layout(int L_s, int H_small, int L_l, int H_large, int n_used
   l.maps_large = align256(per_head * NL);
   l.norms = align256(sizeof(float) * 2 * (NS + NL));   // squared norms, then sums
   l.craw = align256(sizeof(float) * NS * NL);
-  l.total = l.maps_small + l.maps_large + l.norms + l.craw;
+  l.lse_small = align256(sizeof(float) * NS * (size_t)n_used);
+  l.lse_large = align256(sizeof(float) * NL * (size_t)n_used);
+  l.tab_small = align256(seq_tables_bytes(L_s, (int64_t)L_s * l.nb));
+  l.tab_large = align256(seq_tables_bytes(L_l, (int64_t)L_l * l.nb));
+  l.seq_small = align256(sizeof(int32_t) * 2 * (size_t)(L_s + 1));
+  l.seq_large = align256(sizeof(int32_t) * 2 * (size_t)(L_l + 1));
+  l.total = l.maps_small + l.maps_large + l.norms + l.craw + l.lse_small + l.lse_large +
+            l.tab_small + l.tab_large + l.seq_small + l.seq_large;
   return l;
 }
 
@@ -359,6 +369,61 @@ static int launch_maps(const MapsParams& p, cudaStream_t stream) {
   return IAMAP_OK;
 }
 
+// cu[s] = s * n_used (s <= L), tok0[s] = s * n (s < L): the layers of a [L, n, H, d] tensor as
+// sequences of n_used tokens.
+__global__ void hm_seq_kernel(int L, int n, int n_used, int32_t* cu, int32_t* tok0) {
+  for (int s = threadIdx.x; s <= L; s += blockDim.x) {
+    cu[s] = s * n_used;
+    tok0[s] = s * n;
+  }
+}
+
+// Maps of one model on the tensor cores: row statistics (compress stage 1 without masses), then
+// every causal tile of every head written head-major with the maps' sums and squared norms.
+static int maps_tc(const void* q, const void* k, int L, int H, int d, int n, int n_used,
+                   int nb, int64_t tiles, float* lse, char* tab_ws, size_t tab_bytes,
+                   int32_t* seq, __nv_bfloat16* maps, float* norm2, float* sum1,
+                   unsigned int* status, cudaStream_t stream) {
+  std::vector<int32_t> cu_host(L + 1);
+  for (int s = 0; s <= L; ++s) cu_host[s] = s * n_used;
+  CompressArgs c;
+  int rc = make_plan(cu_host.data(), L, kTile, (int64_t)L * n_used, &c.plan);
+  if (rc) return rc;
+  int32_t* cu = seq;
+  int32_t* tok0 = seq + (L + 1);
+  hm_seq_kernel<<<1, 256, 0, stream>>>(L, n, n_used, cu, tok0);
+  IAMAP_LAUNCH_CHECK("hm_seq_kernel");
+  if (seq_tables_bytes(L, c.plan.num_rowblocks) > tab_bytes)
+    return set_error(IAMAP_ERR_WORKSPACE, "head_match: scheduling tables do not fit");
+  c.tab = carve_seq_tables(tab_ws, L, c.plan.num_rowblocks);
+  rc = launch_build_tables(cu, L, kTile, c.plan.max_nb, c.tab, stream);
+  if (rc) return rc;
+  c.q = q;
+  c.k = k;
+  c.cu_seqlens = cu;
+  c.num_seqs = L;
+  c.n = (int64_t)L * n_used;
+  c.n_tok = (int64_t)L * n;
+  c.tok0 = tok0;
+  c.H_s = H;
+  c.d = d;
+  c.tau = 1.f;
+  c.lse = lse;
+  c.mass = nullptr;
+  c.status = status;
+  rc = compress_stats_tc_launch(c, stream);
+  if (rc) return rc;
+  c.lse_in = lse;
+  c.dense = 1;
+  c.dense_tiles = tiles;
+  c.vals = maps;
+  c.capacity = (int64_t)L * H * tiles;
+  c.norm2 = norm2;
+  c.sum1 = sum1;
+  (void)nb;
+  return compress_extract_tc_launch(c, stream);
+}
+
 int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream) {
   const HmLayout l = hm_layout(a.L_s, a.H_small, a.L_l, a.H_large, a.n_used);
   char* ws = static_cast<char*>(a.ws);
@@ -369,6 +434,28 @@ int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream) {
   const int NS = a.L_s * a.H_small, NL = a.L_l * a.H_large;
   IAMAP_CUDA_CHECK(cudaMemsetAsync(norms, 0, l.norms + l.craw, stream));
 
+  // Maps on the tensor cores for prompts of 2048+ tokens. At n_used = 1024 (16 row blocks) both
+  // forms took the same time on a B200 (1.12 vs 1.14 ms per calibration): a CTA of the
+  // tensor-core kernels then has at most 8 key tiles to amortise its set-up over.
+  const bool tc_maps = a.n_used >= 2048 && compress_tc_supported(a.d_small, l.nb) &&
+                       compress_tc_supported(a.d_large, l.nb);
+  if (tc_maps) {
+    char* p = ws + l.maps_small + l.maps_large + l.norms + l.craw;
+    float* lse_s = reinterpret_cast<float*>(p);
+    float* lse_l = reinterpret_cast<float*>(p + l.lse_small);
+    char* tab_s = p + l.lse_small + l.lse_large;
+    char* tab_l = tab_s + l.tab_small;
+    int32_t* seq_s = reinterpret_cast<int32_t*>(tab_l + l.tab_large);
+    int32_t* seq_l = reinterpret_cast<int32_t*>(tab_l + l.tab_large + l.seq_small);
+    int rc = maps_tc(a.q_small, a.k_small, a.L_s, a.H_small, a.d_small, a.n, a.n_used, l.nb,
+                     l.tiles, lse_s, tab_s, l.tab_small, seq_s, maps_small, norms,
+                     norms + NS + NL, a.status, stream);
+    if (!rc)
+      rc = maps_tc(a.q_large, a.k_large, a.L_l, a.H_large, a.d_large, a.n, a.n_used, l.nb,
+                   l.tiles, lse_l, tab_l, l.tab_large, seq_l, maps_large, norms + NS,
+                   norms + NS + NL + NS, a.status, stream);
+    if (rc) return rc;
+  } else {
   MapsParams ps{};
   ps.q = static_cast<const __nv_bfloat16*>(a.q_small);
   ps.k = static_cast<const __nv_bfloat16*>(a.k_small);
@@ -395,6 +482,7 @@ int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream) {
   pl.sum1 = norms + NS + NL + NS;
   rc = a.d_large == 64 ? launch_maps<64>(pl, stream) : launch_maps<128>(pl, stream);
   if (rc) return rc;
+  }
 
   {
     GramTcParams gp{};

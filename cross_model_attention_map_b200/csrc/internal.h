@@ -36,6 +36,16 @@ struct CompressArgs {
   void* vals = nullptr;
   int64_t capacity = 0;
   unsigned int* status = nullptr;
+  // head_match's use of the tensor-core kernels (compress_tc.cu): sequences at token offsets
+  // tok0[s] of q/k tensors holding n_tok tokens (lse and rows are indexed by the packed
+  // cu_seqlens), statistics without masses (mass == nullptr), and the dense head-major output
+  // with per-head sums and squared norms.
+  const int32_t* tok0 = nullptr;
+  int64_t n_tok = 0;
+  int dense = 0;
+  int64_t dense_tiles = 0;
+  float* norm2 = nullptr;
+  float* sum1 = nullptr;
 };
 
 int compress_stats_impl(const CompressArgs& a, cudaStream_t stream);

@@ -430,23 +430,11 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
           if (lane == 0) tc::mbar_arrive(bar_addr(bars, D_EMPTY + gs));
           ++gp;
         }
-        // transpose: position = lane, head = register  ->  16-byte runs of one head. Lanes 2m and
-        // 2m+1 swap one value per head pair, so that each stores one bf16x2 word: positions
-        // (2m, 2m+1) of the even head (even lane) or of the odd head (odd lane).
-        {
-          const bool odd = lane & 1;
-          uint32_t* scr32 = reinterpret_cast<uint32_t*>(scr);
+        // transpose: position = lane, head = register  ->  16-byte runs of one head
 #pragma unroll
-          for (int r = 0; r < 32; r += 2) {
-            if (r < p.NR) {
-              const float mine = __uint_as_float(odd ? v[r + 1] : v[r]);
-              const float send = __uint_as_float(odd ? v[r] : v[r + 1]);
-              const float got = __shfl_xor_sync(0xffffffffu, send, 1);
-              const uint32_t w = odd ? pack_bf16(got, mine) : pack_bf16(mine, got);
-              scr32[(r + (odd ? 1 : 0)) * 16 + (lane >> 1)] = w;
-            }
-          }
-        }
+        for (int r = 0; r < 32; ++r)
+          if (r < p.NR)
+            reinterpret_cast<__nv_bfloat16*>(scr)[r * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[r]));
         __syncwarp();
         const int pos0 = 32 * e;                          // this warp's first position in the chunk
         const int arow = 2 * ch + (pos0 >> 6);            // tile row

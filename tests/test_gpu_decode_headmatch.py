@@ -86,6 +86,19 @@ def test_head_match_small_parity(C, n, n_used, d_small, d_large):
     np.testing.assert_array_equal(arg.reshape(arg_ref.shape), arg_ref)
 
 
+@pytest.mark.parametrize("metric", ["cosine", "pearson"])
+def test_head_match_long_prompt_tensor_core_maps(C, metric):
+    """n_used >= 2048 builds the maps with the tensor-core compress kernels (row statistics, then
+    dense head-major tiles with their sums and norms)."""
+    hm = make_head_match(n=2304, L_s=2, H_small=3, d_small=64, L_l=1, H_large=4,
+                         d_large=128, noise=0.3, seed=38)
+    arg, sim = _run_hm(hm, 2100, metric)
+    assert C.iamap_device_status() == 0
+    S_ref, _ = O.head_match(hm, n_used=2100, metric=metric)
+    np.testing.assert_allclose(sim, S_ref, rtol=0, atol=3e-3)
+    _argmax_matches(arg, S_ref, 6e-3)
+
+
 def test_head_match_calibration_workload(C):
     """n=1024, small 24 x 14 heads d=64, large 8 x 64 heads d=128, noisy zero-padded copies: the
     GPU argmax equals the planted mapping (which the oracle also recovers: oracle pin tests) and
