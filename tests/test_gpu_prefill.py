@@ -96,6 +96,7 @@ def test_tiny_config_full_parity(C):
     ([1000, 130], 12, 10, 128, 0.95, (128, 2.0)),         # d=128, local bias, H_r % 4 != 0
     ([640], 3, 2, 128, 1.0, (0, 0.0)),                    # keep everything
     ([450, 70], 7, 9, 64, 0.3, (16, 2.0)),                # aggressive sparsity
+    ([130, 0, 64, 0], 4, 4, 64, 0.9, (0, 0.0)),           # empty sequences inside the batch
 ])
 def test_varlen_parity(C, seqlens, H_s, H_r, d, tau, bias):
     wl = make_prefill(seqlens, H_s=H_s, d=d, H_r=H_r, d_v=d, B=64, tau=tau, std=1.5, sink=True,
@@ -223,3 +224,11 @@ def test_varlen40k_sampled(C):
     """4 packed sequences 4096/8192/12288/16384, 40 sender heads, 32 receiver heads, tau=0.9."""
     wl = prefill_config("varlen40k")
     _sampled_parity(C, wl, [(0, 63), (1, 5), (2, 191), (3, 0), (3, 255)])
+
+
+def test_sequence_longer_than_16384_tokens(C):
+    """257 row blocks: the compress stages take the mma.sync kernels (the tensor-core statistics
+    keep at most 256 column blocks per row in TMEM); mapped_av stays on the tensor cores."""
+    wl = make_prefill([16448, 300], H_s=2, d=64, H_r=3, d_v=64, B=64, tau=0.9, std=1.5,
+                      sink=True, seed=46)
+    _sampled_parity(C, wl, [(0, 0), (0, 131), (0, 256), (1, 4)])
