@@ -181,11 +181,13 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest x over the ranks (a CPU tensor on gloo, a device tensor on NCCL)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 

@@ -119,3 +119,29 @@ def mapping_consistency(argmax_a, argmax_b, stream=None):
     agree = torch.zeros(1, dtype=torch.int32, device=argmax_a.device)
     C.iamap_mapping_consistency(argmax_a, argmax_b, argmax_a.numel(), agree, stream)
     return agree
+
+
+# ------------------------------------------------------------------------------------------------
+# Several GPUs: head matching split by large layers
+# ------------------------------------------------------------------------------------------------
+
+def shard_range(total, world, rank):
+    """[lo, hi) of `total` items given to `rank` of `world`: contiguous blocks of
+    ceil(total / world), the last ones possibly short or empty."""
+    per = -(-total // world)
+    lo = min(total, rank * per)
+    return lo, min(total, lo + per)
+
+
+def gather_head_mapping(local_argmax, L_l, H_large, group=None):
+    """All ranks' head mappings of their large-layer shards ([hi - lo, H_large] int32 on this
+    rank's device, shards from shard_range) -> the full [L_l, H_large] mapping on every rank, with
+    one all_gather of int32 (the only collective of a sharded calibration)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    per = -(-L_l // world)
+    pad = torch.zeros(per, H_large, dtype=torch.int32, device=local_argmax.device)
+    pad[:local_argmax.shape[0]] = local_argmax.view(-1, H_large)
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    return torch.cat(parts, dim=0)[:L_l]

@@ -1,0 +1,97 @@
+"""The multi-process host paths on CPU: world_size 2 over gloo (no GPU).
+
+- bench.py's barrier and max-over-ranks timing;
+- head matching split by large layers across ranks, reassembled with one all_gather; each
+  rank's shard is computed here by the float64 oracle (the GPU entry point is the same call on
+  the shard's slice of the large model's q, k).
+"""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _init(rank, world, port):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+
+
+def _bench_helpers(rank, world, port, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    _init(rank, world, port)
+    try:
+        bench.barrier(world)
+        out[rank] = bench.max_over_ranks(1.5 + rank, world)
+    finally:
+        dist.destroy_process_group()
+
+
+def _sharded_head_match(rank, world, port, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    import dataclasses
+    import oracle as O
+    from synth import make_head_match
+    from cross_model_attention_map_b200.runner import gather_head_mapping, shard_range
+    _init(rank, world, port)
+    try:
+        hm = make_head_match(n=40, L_s=2, H_small=3, d_small=8, L_l=3, H_large=4, d_large=16,
+                             noise=0.3, seed=51)
+        lo, hi = shard_range(hm.L_l, world, rank)
+        local = dataclasses.replace(hm, L_l=hi - lo, q_large=hm.q_large[lo:hi],
+                                    k_large=hm.k_large[lo:hi])
+        _, arg = O.head_match(local) if hi > lo else (None, np.zeros((0, 4), np.int32))
+        full = gather_head_mapping(torch.from_numpy(np.ascontiguousarray(arg, dtype=np.int32)),
+                                   hm.L_l, hm.H_large)
+        out[rank] = full.numpy().tolist()
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(fn, world=2):
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(fn, args=(world, _free_port(), out), nprocs=world, join=True,
+                           start_method="spawn")
+        return dict(out)
+
+
+def test_shard_range_covers_every_item_once():
+    from cross_model_attention_map_b200.runner import shard_range
+    for total in (0, 1, 7, 8, 9):
+        for world in (1, 2, 3, 8):
+            got = [i for r in range(world) for i in range(*shard_range(total, world, r))]
+            assert got == list(range(total))
+
+
+def test_bench_max_over_ranks_gloo():
+    out = _run(_bench_helpers)
+    assert out == {0: 2.5, 1: 2.5}
+
+
+def test_sharded_head_match_equals_single_process():
+    import oracle as O
+    from synth import make_head_match
+    out = _run(_sharded_head_match)
+    hm = make_head_match(n=40, L_s=2, H_small=3, d_small=8, L_l=3, H_large=4, d_large=16,
+                         noise=0.3, seed=51)
+    _, ref = O.head_match(hm)
+    for rank in (0, 1):
+        np.testing.assert_array_equal(np.array(out[rank]), ref)
