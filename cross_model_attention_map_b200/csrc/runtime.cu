@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "tc_utils.cuh"
 
 namespace iamap {
 
@@ -159,7 +160,48 @@ int launch_build_tables(const int32_t* cu_seqlens, int num_seqs, int B, int32_t 
 
 }  // namespace iamap
 
+namespace iamap {
+
+// One CTA waits on an mbarrier that nothing arrives on, with the kernels' bounded wait and a
+// short limit: the timeout path (status bit, abort flag, orderly return) without a real stall.
+__global__ void selftest_timeout_kernel(unsigned int* status, uint64_t limit_ns, int* gave_up) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = tc::wait_bar_for(smem_u32(&bar), 0, &abort_flag, status, limit_ns);
+    *gave_up = (!ok && abort_flag) ? 1 : 0;
+  }
+}
+
+}  // namespace iamap
+
+namespace iamap {
+
+int selftest_timeout(int limit_us, int* gave_up_dev, cudaStream_t stream) {
+  DeviceContext* c = device_context();
+  if (!c) return IAMAP_ERR_CUDA;
+  selftest_timeout_kernel<<<1, 32, 0, stream>>>(c->status, (uint64_t)limit_us * 1000ull,
+                                                gave_up_dev);
+  IAMAP_LAUNCH_CHECK("selftest_timeout_kernel");
+  return IAMAP_OK;
+}
+
+}  // namespace iamap
+
 using namespace iamap;
+
+extern "C" int iamap_selftest_wait_timeout(int limit_us, int* gave_up, void* stream) {
+  clear_error();
+  if (limit_us < 1 || limit_us > 1000000 || !gave_up)
+    return set_error(IAMAP_ERR_INVALID_ARG, "limit_us must be in [1, 1e6] and gave_up non-null");
+  return selftest_timeout(limit_us, gave_up, static_cast<cudaStream_t>(stream));
+}
 
 extern "C" int iamap_version(void) { return (0 << 16) | 1; }
 

@@ -55,10 +55,10 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
   return ok != 0;
 }
 
-// Waits for the phase of `parity` to complete. Gives up after 2 s (or at once if this CTA already
-// gave up): records IAMAP_DEV_TIMEOUT, sets the CTA's abort flag and returns false.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         unsigned int* status) {
+// Waits for the phase of `parity` to complete. Gives up after limit_ns (or at once if this CTA
+// already gave up): records IAMAP_DEV_TIMEOUT, sets the CTA's abort flag and returns false.
+__device__ __forceinline__ bool wait_bar_for(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned int* status, uint64_t limit_ns) {
   if (*abort_flag) return false;
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -66,13 +66,19 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if ((it & 15u) == 0u) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > 2000000000ull) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         raise_status(status, IAMAP_DEV_TIMEOUT);
         return false;
       }
     }
   }
+}
+
+// The kernels' wait: 2 s.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         unsigned int* status) {
+  return wait_bar_for(bar, parity, abort_flag, status, 2000000000ull);
 }
 
 // Teardown wait: ignores the abort flag (so that asynchronous copies and MMAs still in flight

@@ -69,6 +69,7 @@ _SIGS = {
     "iamap_head_match_metric": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P,
                                      _P, _SZ, _P]),
     "iamap_mapping_consistency": (_I, [_P, _P, _I, _P, _P]),
+    "iamap_selftest_wait_timeout": (_I, [_I, _P, _P]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -250,6 +251,11 @@ def iamap_head_match_metric(q_small, k_small, L_s, H_small, d_small, q_large, k_
         _ptr(q_small), _ptr(k_small), L_s, H_small, d_small, _ptr(q_large), _ptr(k_large), L_l,
         H_large, d_large, n, n_used, metric, _ptr(argmax), _ptr(sim), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def iamap_selftest_wait_timeout(limit_us, gave_up, stream=None):
+    _check("iamap_selftest_wait_timeout", _lib.iamap_selftest_wait_timeout(
+        limit_us, _ptr(gave_up), _stream(stream)))
 
 
 def iamap_mapping_consistency(a, b, n_heads, agree, stream=None):

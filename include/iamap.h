@@ -233,6 +233,14 @@ int iamap_mapped_av_paged_noalloc(const float* p_rows, int ctx_stride, const flo
                                   int H_s, int H_r, int d_v, float* out, void* stream);
 
 /*
+ * Failure-detection self-test: one CTA waits, with the kernels' bounded mbarrier wait but a limit
+ * of limit_us microseconds (1 .. 1e6), on a barrier that nothing arrives on. The wait gives up:
+ * IAMAP_DEV_TIMEOUT is raised in the device status and *gave_up (device int) becomes 1. The
+ * context stays usable. Asynchronous on stream.
+ */
+int iamap_selftest_wait_timeout(int limit_us, int* gave_up, void* stream);
+
+/*
  * Head matching (calibration). q_small / k_small bf16 [L_s, n, H_small, d_small];
  * q_large / k_large bf16 [L_l, n, H_large, d_large]. Each head's map is the causal softmax of
  * q k^T / sqrt(d) over the first n_used tokens (n_used <= n; the prompt truncation tau_t).
