@@ -26,9 +26,9 @@
 // Roles: warps 0, 8, 9, 10 load the sender slices, warp 7 builds W', warps 6, 11, 17, 18 load
 // the V tiles (one receiver head each), one thread of warp 1 issues the mixing MMAs and one
 // thread of warp 12 the P.V MMAs (two issuers: MMA and commit issue costs add up on one thread).
-// Two groups of four warps (2-5 and 13-16) take alternate stored blocks: they read the mixing
-// results out of TMEM, transpose and send them; the first group also writes the output. Every
-// wait is bounded (2 s, then IAMAP_DEV_TIMEOUT).
+// Two groups of four warps (2-5 and 13-16) take the even and the odd chunk pairs of every stored
+// block: they read the mixing results out of TMEM, transpose and send them; the first group also
+// writes the output. Every wait is bounded (2 s, then IAMAP_DEV_TIMEOUT).
 #include <cudaTypedefs.h>
 
 #include <algorithm>
