@@ -48,17 +48,18 @@ class PrefillLayer:
                          b["headmask_dense"], b["row_ptr"], b["col_idx"], b["headmask"],
                          b["val_off"], b["counts"], self.vals, self.capacity, self.ws, stream)
 
-    def mapped_av(self, W, v, stream=None):
+    def mapped_av(self, W, v, stream=None, out=None):
         b = self.bufs
+        out = self.out if out is None else out
         C.iamap_mapped_av_gqa(self.cu, self.cu_host, self.num_seqs, self.n, self.B, self.H_s,
                               b["row_ptr"], b["col_idx"], b["headmask"], b["val_off"], self.vals,
-                              self.capacity, W, self.H_r, self.H_kv, v, self.d_v, self.out,
-                              self.ws, stream)
+                              self.capacity, W, self.H_r, self.H_kv, v, self.d_v, out, self.ws,
+                              stream)
+        return out
 
-    def step(self, q, k, W, v, stream=None):
+    def step(self, q, k, W, v, stream=None, out=None):
         self.compress(q, k, stream)
-        self.mapped_av(W, v, stream)
-        return self.out
+        return self.mapped_av(W, v, stream, out)
 
     def counts(self):
         """(nnz_blocks, nnz_tiles) -- synchronises."""
@@ -145,3 +146,74 @@ def gather_head_mapping(local_argmax, L_l, H_large, group=None):
     parts = [torch.empty_like(pad) for _ in range(world)]
     dist.all_gather(parts, pad, group=group)
     return torch.cat(parts, dim=0)[:L_l]
+
+
+class HostPrefillPipeline:
+    """Prefill steps of one PrefillLayer on host-resident (pinned) inputs, with the upload of the
+    next step's q, k, v, W and the read-back of the previous step's output overlapping the current
+    step's kernels: two device sets of inputs and outputs, one upload and one download stream,
+    the kernels in order on the compute stream. Every step still moves its own inputs in and its
+    own output out."""
+
+    def __init__(self, layer, device="cuda"):
+        self.layer = layer
+        self.up = torch.cuda.Stream(device)
+        self.down = torch.cuda.Stream(device)
+        dev = torch.device(device)
+        n, H_s, d, H_r, H_kv, d_v = layer.n, layer.H_s, layer.d, layer.H_r, layer.H_kv, layer.d_v
+        self.sets = [dict(q=torch.empty(n, H_s, d, dtype=torch.bfloat16, device=dev),
+                          k=torch.empty(n, H_s, d, dtype=torch.bfloat16, device=dev),
+                          v=torch.empty(n, H_kv, d_v, dtype=torch.bfloat16, device=dev),
+                          W=torch.empty(H_r, H_s, dtype=torch.float32, device=dev),
+                          out=torch.empty(n, H_r, d_v, dtype=torch.float32, device=dev))
+                     for _ in range(2)]
+        self.uploaded = [torch.cuda.Event() for _ in range(2)]
+        self.computed = [torch.cuda.Event() for _ in range(2)]
+        self.downloaded = [torch.cuda.Event() for _ in range(2)]
+
+    def bytes_per_step(self):
+        """(host-to-device, device-to-host) bytes of one step."""
+        st = self.sets[0]
+        h2d = sum(st[x].numel() * st[x].element_size() for x in ("q", "k", "v", "W"))
+        return h2d, st["out"].numel() * st["out"].element_size()
+
+    def run(self, host_inputs, host_outputs, stream=None, start_event=None):
+        """host_inputs[i] = (q, k, v, W) pinned CPU tensors of step i; host_outputs[i] the pinned
+        CPU tensor receiving its output (entries may repeat: a buffer is written in step order).
+        Enqueues every step and returns the event recorded on `stream` after the last read-back.
+        start_event (recorded on `stream` by the caller) gates the first upload."""
+        comp = torch.cuda.current_stream() if stream is None else stream
+        n = len(host_inputs)
+
+        def upload(i):
+            s = i % 2
+            with torch.cuda.stream(self.up):
+                if i == 0 and start_event is not None:
+                    self.up.wait_event(start_event)
+                if i >= 2:
+                    self.up.wait_event(self.computed[s])    # step i - 2 has read set s
+                for name, h in zip(("q", "k", "v", "W"), host_inputs[i]):
+                    self.sets[s][name].copy_(h, non_blocking=True)
+                self.uploaded[s].record(self.up)
+
+        if n:
+            upload(0)
+        for i in range(n):
+            s = i % 2
+            st = self.sets[s]
+            if i + 1 < n:
+                upload(i + 1)
+            comp.wait_event(self.uploaded[s])
+            if i >= 2:
+                comp.wait_event(self.downloaded[s])          # step i - 2's output was read back
+            self.layer.step(st["q"], st["k"], st["W"], st["v"], comp, out=st["out"])
+            self.computed[s].record(comp)
+            with torch.cuda.stream(self.down):
+                self.down.wait_event(self.computed[s])
+                host_outputs[i].copy_(st["out"], non_blocking=True)
+                self.downloaded[s].record(self.down)
+        done = torch.cuda.Event(enable_timing=True)
+        if n:
+            comp.wait_event(self.downloaded[(n - 1) % 2])
+        done.record(comp)
+        return done

@@ -232,3 +232,26 @@ def test_sequence_longer_than_16384_tokens(C):
     wl = make_prefill([16448, 300], H_s=2, d=64, H_r=3, d_v=64, B=64, tau=0.9, std=1.5,
                       sink=True, seed=46)
     _sampled_parity(C, wl, [(0, 0), (0, 131), (0, 256), (1, 4)])
+
+
+def test_host_pipeline_equals_direct_steps(C):
+    """HostPrefillPipeline (uploads and read-backs overlapping the kernels of other steps) gives
+    every step exactly the output of a direct step on the same inputs."""
+    from cross_model_attention_map_b200.runner import HostPrefillPipeline, PrefillLayer
+    wls = [make_prefill([300, 200], H_s=4, d=64, H_r=4, d_v=64, B=64, tau=0.9, seed=s)
+           for s in (71, 72, 73)]
+    layer = PrefillLayer(wls[0].seqlens, 4, 64, 4, 64, 0.9)
+
+    def pinned(x):
+        return x.cpu().pin_memory()
+
+    ins = [tuple(pinned(t) for t in upload_prefill(wl)) for wl in wls]
+    outs = [torch.empty(layer.out.shape, dtype=torch.float32).pin_memory() for _ in wls]
+    pipe = HostPrefillPipeline(layer)
+    pipe.run(ins, outs).synchronize()
+    assert C.iamap_device_status() == 0
+    for wl, o in zip(wls, outs):
+        q, k, v, W = upload_prefill(wl)
+        ref = layer.step(q, k, W, v).cpu()
+        torch.cuda.synchronize()
+        assert torch.equal(o, ref)
