@@ -18,7 +18,12 @@
  *                Different-scale LLMs" notes, Method section 4, decode bullet.)
  *   head_match   IAM's calibration: cosine similarity of flattened causal attention maps of every
  *                large-model head with every small-model head, then the most similar small head
- *                per large head. (IAM notes, Method sections 1 and 4.)
+ *                per large head. (IAM notes, Method sections 1 and 4.) Variants: Pearson and
+ *                Euclidean similarity (section 1), the agreement count of two mappings
+ *                (section 3).
+ *   *_gqa        mapped_av / mapped_av_paged with grouped receiver values: H_kv value heads,
+ *                receiver head r reads value head r / (H_r / H_kv).
+ *   iamap_selftest_wait_timeout  exercises the bounded-wait failure path on the GPU.
  *
  * Conventions (all entry points):
  *   - Return 0 (IAMAP_OK) or a negative IAMAP_ERR_* code; iamap_last_error() gives a
@@ -35,7 +40,7 @@
  *
  * Layouts:
  *   q, k      bf16 [n, H_s, d]     token-major, packed sequences (cu_seqlens, int32 [S+1])
- *   v         bf16 [n, H_r, d_v]
+ *   v         bf16 [n, H_r, d_v]   ([n, H_kv, d_v] for the *_gqa entry points)
  *   W         fp32 [H_r, H_s]      row r mixes the sender heads for receiver head r
  *   lse       fp32 [H_s, n]        natural-log row log-sum-exp of the sender's scaled logits
  *   Causal blocks: sequence s has nb_s = ceil(L_s / B) row blocks; row block I has column blocks
