@@ -85,3 +85,21 @@ def test_workspace_queries(lib):
     assert lib.iamap_compress_workspace_bytes(4, 640) > 640 * 8
     assert lib.iamap_head_match_workspace_bytes(24, 14, 8, 64, 1024) > 848 * 136 * 8192
     assert lib.iamap_mapped_av_paged_workspace_bytes(4, 64, 128, 8704, 16) > 0
+
+
+def test_host_validation_of_variants(lib):
+    """The metric, grouped-value, consistency and self-test entry points refuse bad arguments
+    on the host."""
+    raw = lib._lib
+    rc = raw.iamap_head_match_metric(None, None, 1, 1, 64, None, None, 1, 1, 128, 8, 8, 7, None,
+                                     None, None, 0, None)
+    assert rc == -1 and "metric" in lib.iamap_last_error()
+    rc = raw.iamap_mapped_av_gqa(None, None, 1, 64, 64, 4, None, None, None, None, None, 0, None,
+                                 8, 3, None, 64, None, None, 0, None)
+    assert rc == -1 and "divide" in lib.iamap_last_error()
+    rc = raw.iamap_mapped_av_paged_gqa(None, 0, None, None, 0, None, 0, 16, None, None, 1, 1, 8,
+                                       3, 64, None, None, 0, None)
+    assert rc == -1 and "divide" in lib.iamap_last_error()
+    assert raw.iamap_mapping_consistency(None, None, 4, None, None) == -1
+    assert raw.iamap_selftest_wait_timeout(0, None, None) == -1
+    assert raw.iamap_selftest_wait_timeout(2_000_000, None, None) == -1
