@@ -19,4 +19,7 @@ from .workloads import (  # noqa: F401
     prefill_config,
     head_match_config,
     decode_config,
+    PrefixWorkload,
+    make_prefix_requests,
+    prefix_config,
 )

@@ -16,6 +16,8 @@ Workloads (one per configuration of the benchmark description):
                  each large head a noisy zero-padded copy of a uniformly drawn small head
 * decode         batch 4, context 8704, sender 14 heads, receiver 64 heads d_v=128, one-hot
                  W, V cache in 16-token pages under a random page table
+* prefix index   token ids of the varlen prompts as the cached set, 16 prompts sharing seeded
+                 prefixes with them (block boundaries and mid-block), uniform over a 151936 vocab
 """
 
 from __future__ import annotations
@@ -244,3 +246,73 @@ def make_decode(batch=4, ctx=8704, H_s=14, H_r=64, d_v=128, page_size=16, sink_w
 
 def decode_config(seed: int = 0) -> DecodeWorkload:
     return make_decode(seed=seed)
+
+
+# ----------------------------------------------------------------------------------------------
+# Token ids for the prefix-hash block index
+# ----------------------------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class PrefixWorkload:
+    B: int
+    salt: int
+    cached_tokens: np.ndarray   # int32, packed sequences already in the index
+    cached_cu: np.ndarray       # int32 [S_c + 1]
+    query_tokens: np.ndarray    # int32, packed prompts looked up
+    query_cu: np.ndarray        # int32 [S_q + 1]
+    shared: list                # per prompt: (cached sequence it copies from or -1, tokens copied)
+
+
+def _pack(seqs):
+    cu = np.zeros(len(seqs) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum([len(x) for x in seqs])
+    toks = np.concatenate(seqs).astype(np.int32) if seqs else np.zeros(0, np.int32)
+    return toks, cu
+
+
+def make_prefix_requests(cached_lens, query_lens, B=64, vocab=151936, seed=0,
+                         p_fresh=0.2) -> PrefixWorkload:
+    """Draw order: salt, cached sequences, then per prompt its source, shared length and tokens.
+
+    Token ids are uniform in [0, vocab). Cached sequence i > 0 copies a prefix of a uniformly
+    drawn earlier cached sequence with probability 1/2 (so the cached set holds repeated prefix
+    blocks). Each prompt copies the first m tokens of a uniformly drawn cached sequence (with
+    probability 1 - p_fresh), m uniform in [0, min(lengths)], every third one rounded down to a
+    multiple of B, and then differs at token m (when m is shorter than the prompt).
+    """
+    rng = np.random.default_rng(seed)
+    salt = int(rng.integers(0, 2**63 - 1, dtype=np.int64))
+    cached = []
+    for i, L in enumerate(cached_lens):
+        x = rng.integers(0, vocab, size=int(L), dtype=np.int64).astype(np.int32)
+        if i > 0 and rng.random() < 0.5:
+            src = cached[int(rng.integers(0, i))]
+            m = int(rng.integers(0, min(len(src), len(x)) + 1))
+            x[:m] = src[:m]
+        cached.append(x)
+    queries, shared = [], []
+    for j, L in enumerate(query_lens):
+        x = rng.integers(0, vocab, size=int(L), dtype=np.int64).astype(np.int32)
+        if cached and rng.random() >= p_fresh:
+            c = int(rng.integers(0, len(cached)))
+            m = int(rng.integers(0, min(len(cached[c]), len(x)) + 1))
+            if j % 3 == 0:
+                m -= m % B
+            x[:m] = cached[c][:m]
+            if m < len(x) and m < len(cached[c]):
+                x[m] = (cached[c][m] + 1 + int(rng.integers(0, vocab - 1))) % vocab
+            shared.append((c, m))
+        else:
+            shared.append((-1, 0))
+        queries.append(x)
+    ct, ccu = _pack(cached)
+    qt, qcu = _pack(queries)
+    return PrefixWorkload(B=B, salt=salt, cached_tokens=ct, cached_cu=ccu, query_tokens=qt,
+                          query_cu=qcu, shared=shared)
+
+
+def prefix_config(seed: int = 0) -> PrefixWorkload:
+    """The packed prompts of the varlen prefill workload (4096/8192/12288/16384 tokens) as the
+    cached set, and 16 prompts of those lengths (four each) looked up against it."""
+    lens = [4096, 8192, 12288, 16384]
+    return make_prefix_requests(lens, lens * 4, seed=seed)

@@ -2,7 +2,7 @@
 
 Small workloads are compared element by element over everything the library writes: lse, block
 masses, per-head kept sets (bit-exact except near-threshold blocks), the union BSR index, every
-stored bf16 tile, and the output. The output is judged against the oracle evaluated on the GPU's
+stored bf16 tile, and the output. The output is compared with the oracle evaluated on the GPU's
 own kept sets (so a near-threshold flip is not mistaken for a kernel error) and, where no flip
 happened, against the oracle's own kept sets too. The full-size workloads are checked on sampled
 row blocks in the launch configuration the benchmark times.
