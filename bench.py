@@ -11,7 +11,7 @@ are resident in HBM when the timed region starts; Q+K (840 MB) and the block-spa
 
 Other configs (for measurement of the other kernels): ``tiny``, ``prefill8k``, ``headmatch``
 (head_match, n=1024, 24x14 small / 8x64 large heads), ``decode`` (paged decode, batch 4,
-context 8704).
+context 8704), ``prefixindex`` (prefix-hash block index: publish and look up prompts).
 
 Multi-GPU (torchrun): every rank runs its own full batch (independent problems, no data-path
 collective, weak scaling); rank 0 prints value = tokens of all ranks / max time over ranks.
@@ -52,6 +52,9 @@ CONFIG_TEXT = {
                   "d=128, planted noisy copies; head_match"),
     "decode": ("decode: batch 4, q_len 1, context 8704, sender 14 heads, receiver 64 heads "
                "d_v=128, one-hot W, 16-token pages; mapped_av_paged"),
+    "prefixindex": ("prefixindex: publish the 4 varlen prompts (40960 tokens, 640 blocks of 64) "
+                    "into an empty 4096-slot prefix-hash index, then look up 16 prompts "
+                    "(163840 tokens, 2560 blocks) sharing seeded prefixes with them"),
 }
 
 
@@ -502,9 +505,127 @@ def bench_headmatch(args, world, rank, local, peaks):
     }, hm
 
 
+def bench_prefixindex(args, world, rank, local, peaks):
+    import torch
+    from synth import prefix_config
+    from cross_model_attention_map_b200 import iamap as C
+    from cross_model_attention_map_b200.runner import PrefixIndex
+
+    dev = torch.device("cuda", local)
+    w = prefix_config(seed=rank)
+    idx = PrefixIndex(1 << 12, B=w.B, salt=w.salt, device=dev)
+    ct = torch.from_numpy(w.cached_tokens).to(dev)
+    qt = torch.from_numpy(w.query_tokens).to(dev)
+    ccu, qcu = torch.from_numpy(w.cached_cu).to(dev), torch.from_numpy(w.query_cu).to(dev)
+    nc = C.iamap_prefix_num_keys(w.cached_cu, len(w.cached_cu) - 1, w.B)
+    nq = C.iamap_prefix_num_keys(w.query_cu, len(w.query_cu) - 1, w.B)
+    ckeys = torch.empty(nc, dtype=torch.int64, device=dev)
+    ccu_k = torch.empty(len(w.cached_cu), dtype=torch.int64, device=dev)
+    qkeys = torch.empty(nq, dtype=torch.int64, device=dev)
+    qcu_k = torch.empty(len(w.query_cu), dtype=torch.int64, device=dev)
+    locs = torch.arange(nc, dtype=torch.int64, device=dev)
+    stored = torch.empty(nc, dtype=torch.int64, device=dev)
+    found = torch.empty(nq, dtype=torch.int64, device=dev)
+    hits = torch.empty(len(w.query_cu) - 1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    stream = torch.cuda.current_stream()
+    S_c, S_q = len(w.cached_cu) - 1, len(w.query_cu) - 1
+
+    def step(e=None):
+        if e:
+            e[0].record(stream)
+        C.iamap_prefix_index_clear(idx.table_keys, idx.table_vals, idx.capacity, stream)
+        C.iamap_prefix_keys(ct, ct.numel(), ccu, S_c, w.B, w.salt, ckeys, nc, ccu_k, stream)
+        C.iamap_prefix_insert(ckeys, locs, nc, idx.table_keys, idx.table_vals, idx.capacity,
+                              stored, stream)
+        if e:
+            e[1].record(stream)
+        C.iamap_prefix_keys(qt, qt.numel(), qcu, S_q, w.B, w.salt, qkeys, nq, qcu_k, stream)
+        if e:
+            e[2].record(stream)
+        C.iamap_prefix_lookup(qkeys, nq, qcu_k, S_q, idx.table_keys, idx.table_vals,
+                              idx.capacity, found, hits, stream)
+        if e:
+            e[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.start()
+    for e in evs:
+        flush.zero_()            # L2 flush outside the timed events
+        step(e)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    assert C.iamap_device_status(stream) == 0
+    ms = max_over_ranks(sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps, world)
+    t_pub = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    t_qkeys = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    t_look = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    tokens = ct.numel() + qt.numel()
+    # prompt keys kernel: token ids read (4 B), keys written (8 B), offsets (8 B per sequence)
+    key_bytes = 4.0 * qt.numel() + 8.0 * nq + 8.0 * (S_q + 1)
+    gbs = key_bytes / (t_qkeys * 1e-3) / 1e9
+    return {
+        "metric": "prefix-index prompt tokens/s (publish + look up, chained 64-token blocks)",
+        "value": round(tokens * world / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+        "data": "synthetic", "config": {"workload": CONFIG_TEXT["prefixindex"],
+                                        "l2": "256 MB buffer written between timed steps",
+                                        "ms_publish": round(t_pub, 4),
+                                        "ms_prompt_keys": round(t_qkeys, 4),
+                                        "ms_lookup": round(t_look, 4)},
+        "roofline": {"kernel": "prefix_keys (16 prompts)", "bound": "hbm",
+                     "achieved": round(gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / peaks["hbm_gbs"], 5), "traffic": None},
+        "clocks": clocks, "gpu_launches": 5 * args.steps,
+    }, w
+
+
+def oracle_prefix_step(w):
+    """One oracle pass of the prefix-index step (publish the cached prompts, look up the others):
+    (tokens/s, seconds)."""
+    from oracle import prefix_index as px
+    t0 = time.perf_counter()
+    ck, _ = px.prefix_keys(w.cached_tokens, w.cached_cu, w.B, w.salt)
+    idx = px.PrefixIndex()
+    idx.insert(ck, np.arange(len(ck), dtype=np.int64))
+    qk, q_cu = px.prefix_keys(w.query_tokens, w.query_cu, w.B, w.salt)
+    px.prefix_hits(idx.lookup(qk), q_cu)
+    dt = time.perf_counter() - t0
+    return (len(w.cached_tokens) + len(w.query_tokens)) / dt, dt
+
+
 def reference_arm(args):
     """The float64 oracle on the host cores, same metric and unit, bounded sample per step."""
     from synth import prefill_config
+    if args.config == "prefixindex":
+        from synth import prefix_config
+        w = prefix_config()
+        for _ in range(args.warmup):
+            oracle_prefix_step(w)
+        vals = [oracle_prefix_step(w)[0] for _ in range(args.steps)]
+        value = statistics.mean(vals)
+        tokens = len(w.cached_tokens) + len(w.query_tokens)
+        print(json.dumps({
+            "impl": "reference",
+            "metric": "prefix-index prompt tokens/s (publish + look up, chained 64-token blocks)",
+            "value": round(value, 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * tokens / value, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+            "data": "synthetic", "config": {"workload": CONFIG_TEXT["prefixindex"]},
+            "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": 1,
+                             "kind": "oracle", "sample": "the whole workload per step"},
+            "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }))
+        return
     if args.config not in ("varlen40k", "prefill8k", "tiny"):
         print(json.dumps({"impl": "reference", "unavailable":
                           "reference arm implemented for the prefill workloads only"}))
@@ -558,6 +679,8 @@ def main():
         line, wl = bench_prefill(args, world, rank, local, peaks)
     elif args.config == "decode":
         line, wl = bench_decode(args, world, rank, local, peaks)
+    elif args.config == "prefixindex":
+        line, wl = bench_prefixindex(args, world, rank, local, peaks)
     else:
         line, wl = bench_headmatch(args, world, rank, local, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config in (
@@ -565,6 +688,11 @@ def main():
         v, rows, dt, text = oracle_sample_prefill(wl, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(v, 2), "unit": "tokens/s", "cores": cores(),
                                 "kind": "oracle", "sample": text + " in %.1f s" % dt}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "prefixindex":
+        v, dt = oracle_prefix_step(wl)
+        line["cpu_baseline"] = {"value": round(v, 1), "unit": "tokens/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": "the whole workload, one pass in %.1f s" % dt}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

@@ -358,3 +358,93 @@ extern "C" int iamap_head_match_metric(const void* q_small, const void* k_small,
   a.status = ctx->status;
   return head_match_impl(a, static_cast<cudaStream_t>(stream));
 }
+
+// ------------------------------------------------------------------------------------------------
+// Prefix-hash block index
+// ------------------------------------------------------------------------------------------------
+
+namespace {
+
+constexpr int64_t kMaxIndexCapacity = int64_t(1) << 40;
+constexpr int kMaxKeyBlock = 4096;
+
+int check_capacity(const void* table_keys, const void* table_vals, int64_t capacity) {
+  if (!table_keys || !table_vals) return set_error(IAMAP_ERR_INVALID_ARG, "null table pointer");
+  if (capacity < 1 || capacity > kMaxIndexCapacity || (capacity & (capacity - 1)) != 0)
+    return set_error(IAMAP_ERR_INVALID_ARG, "capacity must be a power of two in [1, 2^40]");
+  return IAMAP_OK;
+}
+
+}  // namespace
+
+extern "C" int iamap_prefix_num_keys(const int32_t* cu_seqlens_host, int num_seqs, int B,
+                                     int64_t* num_keys) {
+  clear_error();
+  if (!cu_seqlens_host || !num_keys) return set_error(IAMAP_ERR_INVALID_ARG, "null pointer");
+  if (num_seqs < 1 || B < 1) return set_error(IAMAP_ERR_INVALID_ARG, "need num_seqs >= 1, B >= 1");
+  if (cu_seqlens_host[0] < 0)
+    return set_error(IAMAP_ERR_INVALID_ARG, "cu_seqlens_host[0] must be >= 0");
+  int64_t t = 0;
+  for (int s = 0; s < num_seqs; ++s) {
+    const int64_t L = (int64_t)cu_seqlens_host[s + 1] - cu_seqlens_host[s];
+    if (L < 0) return set_error(IAMAP_ERR_INVALID_ARG, "cu_seqlens_host decreases at %d", s);
+    t += L / B;
+  }
+  *num_keys = t;
+  return IAMAP_OK;
+}
+
+extern "C" int iamap_prefix_keys(const int32_t* tokens, int64_t n, const int32_t* cu_seqlens,
+                                 int num_seqs, int B, uint64_t salt, uint64_t* keys,
+                                 int64_t keys_capacity, int64_t* key_cu, void* stream) {
+  clear_error();
+  if (!cu_seqlens || !key_cu) return set_error(IAMAP_ERR_INVALID_ARG, "null pointer");
+  if (n < 0 || num_seqs < 1 || keys_capacity < 0)
+    return set_error(IAMAP_ERR_INVALID_ARG, "need n >= 0, num_seqs >= 1, keys_capacity >= 0");
+  if (n > 0 && !tokens) return set_error(IAMAP_ERR_INVALID_ARG, "tokens is null");
+  if (keys_capacity > 0 && !keys) return set_error(IAMAP_ERR_INVALID_ARG, "keys is null");
+  if (B < 1 || B > kMaxKeyBlock)
+    return set_error(IAMAP_ERR_INVALID_ARG, "B must be in [1, %d]", kMaxKeyBlock);
+  return prefix_keys_launch(tokens, n, cu_seqlens, num_seqs, B, salt, keys, keys_capacity, key_cu,
+                            static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int iamap_prefix_index_clear(uint64_t* table_keys, int64_t* table_vals,
+                                        int64_t capacity, void* stream) {
+  clear_error();
+  int rc = check_capacity(table_keys, table_vals, capacity);
+  if (rc) return rc;
+  if (!device_context()) return IAMAP_ERR_CUDA;
+  return prefix_clear_launch(table_keys, table_vals, capacity, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int iamap_prefix_insert(const uint64_t* keys, const int64_t* values, int64_t count,
+                                   uint64_t* table_keys, int64_t* table_vals, int64_t capacity,
+                                   int64_t* stored, void* stream) {
+  clear_error();
+  int rc = check_capacity(table_keys, table_vals, capacity);
+  if (rc) return rc;
+  if (count < 0 || count > kMaxIndexCapacity)
+    return set_error(IAMAP_ERR_INVALID_ARG, "count must be in [0, 2^40]");
+  if (count > 0 && (!keys || !values || !stored))
+    return set_error(IAMAP_ERR_INVALID_ARG, "null pointer");
+  return prefix_insert_launch(keys, values, count, table_keys, table_vals, capacity, stored,
+                              static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int iamap_prefix_lookup(const uint64_t* keys, int64_t count, const int64_t* key_cu,
+                                   int num_seqs, const uint64_t* table_keys,
+                                   const int64_t* table_vals, int64_t capacity, int64_t* found,
+                                   int32_t* hit_blocks, void* stream) {
+  clear_error();
+  int rc = check_capacity(table_keys, table_vals, capacity);
+  if (rc) return rc;
+  if (count < 0 || count > kMaxIndexCapacity)
+    return set_error(IAMAP_ERR_INVALID_ARG, "count must be in [0, 2^40]");
+  if (count > 0 && (!keys || !found)) return set_error(IAMAP_ERR_INVALID_ARG, "null pointer");
+  if ((key_cu == nullptr) != (hit_blocks == nullptr))
+    return set_error(IAMAP_ERR_INVALID_ARG, "key_cu and hit_blocks go together");
+  if (key_cu && num_seqs < 1) return set_error(IAMAP_ERR_INVALID_ARG, "num_seqs must be >= 1");
+  return prefix_lookup_launch(keys, count, key_cu, num_seqs, table_keys, table_vals, capacity,
+                              found, hit_blocks, static_cast<cudaStream_t>(stream));
+}

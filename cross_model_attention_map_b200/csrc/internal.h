@@ -126,4 +126,18 @@ int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream);
 int consistency_impl(const int32_t* a, const int32_t* b, int n, int32_t* agree,
                      cudaStream_t stream);
 
+// Prefix-hash block index (prefix_index.cu).
+int prefix_keys_launch(const int32_t* tokens, int64_t n, const int32_t* cu, int num_seqs, int B,
+                       uint64_t salt, uint64_t* keys, int64_t keys_capacity, int64_t* key_cu,
+                       cudaStream_t stream);
+int prefix_clear_launch(uint64_t* table_keys, int64_t* table_vals, int64_t capacity,
+                        cudaStream_t stream);
+int prefix_insert_launch(const uint64_t* keys, const int64_t* values, int64_t count,
+                         uint64_t* table_keys, int64_t* table_vals, int64_t capacity,
+                         int64_t* stored, cudaStream_t stream);
+int prefix_lookup_launch(const uint64_t* keys, int64_t count, const int64_t* key_cu,
+                         int num_seqs, const uint64_t* table_keys, const int64_t* table_vals,
+                         int64_t capacity, int64_t* found, int32_t* hit_blocks,
+                         cudaStream_t stream);
+
 }  // namespace iamap

@@ -38,6 +38,7 @@ _I = ctypes.c_int
 _I64 = ctypes.c_int64
 _F = ctypes.c_float
 _SZ = ctypes.c_size_t
+_U64 = ctypes.c_uint64
 
 _SIGS = {
     "iamap_version": (_I, []),
@@ -70,6 +71,11 @@ _SIGS = {
                                      _P, _SZ, _P]),
     "iamap_mapping_consistency": (_I, [_P, _P, _I, _P, _P]),
     "iamap_selftest_wait_timeout": (_I, [_I, _P, _P]),
+    "iamap_prefix_num_keys": (_I, [_P, _I, _I, ctypes.POINTER(_I64)]),
+    "iamap_prefix_keys": (_I, [_P, _I64, _P, _I, _I, _U64, _P, _I64, _P, _P]),
+    "iamap_prefix_index_clear": (_I, [_P, _P, _I64, _P]),
+    "iamap_prefix_insert": (_I, [_P, _P, _I64, _P, _P, _I64, _P, _P]),
+    "iamap_prefix_lookup": (_I, [_P, _I64, _P, _I, _P, _P, _I64, _P, _P, _P]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -269,6 +275,41 @@ def iamap_head_match(q_small, k_small, L_s, H_small, d_small, q_large, k_large, 
         _ptr(q_small), _ptr(k_small), L_s, H_small, d_small, _ptr(q_large), _ptr(k_large), L_l,
         H_large, d_large, n, n_used, _ptr(argmax), _ptr(sim), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def iamap_prefix_num_keys(cu_seqlens_host, num_seqs, B) -> int:
+    cu, _keep = _host_i32(cu_seqlens_host)
+    out = _I64(0)
+    _check("iamap_prefix_num_keys", _lib.iamap_prefix_num_keys(cu, num_seqs, B,
+                                                               ctypes.byref(out)))
+    return out.value
+
+
+def iamap_prefix_keys(tokens, n, cu_seqlens, num_seqs, B, salt, keys, keys_capacity, key_cu,
+                      stream=None):
+    """keys: a uint64 buffer carried as an int64 tensor (same bits)."""
+    _check("iamap_prefix_keys", _lib.iamap_prefix_keys(
+        _ptr(tokens), n, _ptr(cu_seqlens), num_seqs, B, int(salt) & (2**64 - 1), _ptr(keys),
+        keys_capacity, _ptr(key_cu), _stream(stream)))
+
+
+def iamap_prefix_index_clear(table_keys, table_vals, capacity, stream=None):
+    _check("iamap_prefix_index_clear", _lib.iamap_prefix_index_clear(
+        _ptr(table_keys), _ptr(table_vals), capacity, _stream(stream)))
+
+
+def iamap_prefix_insert(keys, values, count, table_keys, table_vals, capacity, stored,
+                        stream=None):
+    _check("iamap_prefix_insert", _lib.iamap_prefix_insert(
+        _ptr(keys), _ptr(values), count, _ptr(table_keys), _ptr(table_vals), capacity,
+        _ptr(stored), _stream(stream)))
+
+
+def iamap_prefix_lookup(keys, count, key_cu, num_seqs, table_keys, table_vals, capacity, found,
+                        hit_blocks, stream=None):
+    _check("iamap_prefix_lookup", _lib.iamap_prefix_lookup(
+        _ptr(keys), count, _ptr(key_cu), num_seqs, _ptr(table_keys), _ptr(table_vals), capacity,
+        _ptr(found), _ptr(hit_blocks), _stream(stream)))
 
 
 # ------------------------------------------------------------------------------------------------

@@ -122,6 +122,51 @@ def mapping_consistency(argmax_a, argmax_b, stream=None):
     return agree
 
 
+class PrefixIndex:
+    """A device prefix-hash index of stored map blocks: `capacity` slots (a power of two) of
+    uint64 keys (carried as int64 tensors) and int64 locations, keys made with `salt` (one salt
+    per sender layer or model)."""
+
+    def __init__(self, capacity, B=64, salt=0xCBF29CE484222325, device="cuda"):
+        self.capacity, self.B, self.salt = int(capacity), int(B), int(salt)
+        self.table_keys = torch.empty(self.capacity, dtype=torch.int64, device=device)
+        self.table_vals = torch.empty(self.capacity, dtype=torch.int64, device=device)
+        self.device = device
+        self.clear()
+
+    def clear(self, stream=None):
+        C.iamap_prefix_index_clear(self.table_keys, self.table_vals, self.capacity, stream)
+
+    def keys(self, tokens, cu_seqlens, cu_seqlens_host, stream=None):
+        """(keys int64 [num_keys], key_cu int64 [num_seqs + 1]) of packed prompts."""
+        num_seqs = len(cu_seqlens_host) - 1
+        nk = C.iamap_prefix_num_keys(cu_seqlens_host, num_seqs, self.B)
+        keys = torch.empty(max(nk, 1), dtype=torch.int64, device=self.device)
+        key_cu = torch.empty(num_seqs + 1, dtype=torch.int64, device=self.device)
+        C.iamap_prefix_keys(tokens, tokens.numel(), cu_seqlens, num_seqs, self.B, self.salt, keys,
+                            nk, key_cu, stream)
+        return keys[:nk], key_cu
+
+    def insert(self, keys, values, stream=None):
+        """Locations now stored for `keys` (int64 [count]); -1 where no slot was found."""
+        stored = torch.empty(max(keys.numel(), 1), dtype=torch.int64, device=self.device)
+        C.iamap_prefix_insert(keys, values, keys.numel(), self.table_keys, self.table_vals,
+                              self.capacity, stored, stream)
+        return stored[:keys.numel()]
+
+    def lookup(self, keys, key_cu=None, stream=None):
+        """(found int64 [count], hit_blocks int32 [num_seqs] or None)."""
+        found = torch.empty(max(keys.numel(), 1), dtype=torch.int64, device=self.device)
+        hits = None
+        num_seqs = 0
+        if key_cu is not None:
+            num_seqs = key_cu.numel() - 1
+            hits = torch.empty(num_seqs, dtype=torch.int32, device=self.device)
+        C.iamap_prefix_lookup(keys, keys.numel(), key_cu, num_seqs, self.table_keys,
+                              self.table_vals, self.capacity, found, hits, stream)
+        return found[:keys.numel()], hits
+
+
 # ------------------------------------------------------------------------------------------------
 # Several GPUs: head matching split by large layers
 # ------------------------------------------------------------------------------------------------

@@ -23,6 +23,10 @@
  *                (section 3).
  *   *_gqa        mapped_av / mapped_av_paged with grouped receiver values: H_kv value heads,
  *                receiver head r reads value head r / (H_r / H_kv).
+ *   prefix index the prefix-hash index of stored map blocks: chained FNV-1a-64 keys of every full
+ *                block of a prompt, insert of (key, location) pairs into a device hash table,
+ *                lookup of a prompt's blocks and of its longest cached prefix. (MapFlow news
+ *                page, storage-and-execution part, second component.)
  *   iamap_selftest_wait_timeout  exercises the bounded-wait failure path on the GPU.
  *
  * Conventions (all entry points):
@@ -35,8 +39,9 @@
  *   - The library keeps one lazily created context per device: a device status word that kernels
  *     set on a detected error (capacity exceeded, bounded wait expired, malformed index). Read and
  *     clear it with iamap_device_status.
- *   - Only block size B = 64 is implemented (IAMAP_ERR_UNSUPPORTED otherwise). Head dims d, d_v
- *     must be 64 or 128. Sender heads H_s <= 64 (one bit per head in the head masks).
+ *   - Only block size B = 64 is implemented for the maps (IAMAP_ERR_UNSUPPORTED otherwise; the
+ *     prefix index takes any B in 1..4096). Head dims d, d_v must be 64 or 128. Sender heads
+ *     H_s <= 64 (one bit per head in the head masks).
  *
  * Layouts:
  *   q, k      bf16 [n, H_s, d]     token-major, packed sequences (cu_seqlens, int32 [S+1])
@@ -280,6 +285,74 @@ int iamap_head_match_metric(const void* q_small, const void* k_small, int L_s, i
  */
 int iamap_mapping_consistency(const int32_t* a, const int32_t* b, int n_heads, int32_t* agree,
                               void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Prefix-hash block index ("PKU MapFlow: cross-model attention map reuse" news page, storage-
+ * and-execution part, second component: stored map blocks are located through a prefix hash
+ * index whose keys carry the preceding context; one sender state can serve several receivers).
+ *
+ * Block b of a packed sequence is tokens [b*B, (b+1)*B) (full blocks only; with B = 64 these are
+ * the map's row blocks). Its digest is FNV-1a-64 (offset basis 0xcbf29ce484222325, prime
+ * 0x100000001b3) of its token ids as 4-byte little-endian integers; its prefix key is the
+ * FNV-1a-64 state after absorbing, from `salt`, the 8-byte little-endian digests of blocks 0..b.
+ * The key therefore changes with any token before the block's end. Pick one salt per sender
+ * layer (or model) so that entries of different layers never share a key.
+ *
+ * The index is an open-addressing table owned by the caller: table_keys (uint64) and table_vals
+ * (int64 locations, e.g. the first tile of the row block's stored blocks), `capacity` entries,
+ * capacity a power of two in [1, 2^40]. The all-ones key marks an empty slot and is never stored.
+ * A key lives within min(capacity, 1024) slots of its home slot (linear probing); keep the load
+ * factor below about 0.7. Entries are never removed (clear the table to start over). Inserts and
+ * lookups on one table must be ordered (same stream, or events): they are not atomic with
+ * respect to each other.
+ * ------------------------------------------------------------------------------------------- */
+
+/*
+ * Number of prefix keys (full blocks) of packed sequences, from host cu_seqlens.
+ * Errors: IAMAP_ERR_INVALID_ARG for a null pointer, num_seqs < 1, B < 1 or decreasing offsets.
+ */
+int iamap_prefix_num_keys(const int32_t* cu_seqlens_host, int num_seqs, int B,
+                          int64_t* num_keys);
+
+/*
+ * Prefix keys of every full block of the packed sequences.
+ *   tokens      int32 [n] device, token ids packed by cu_seqlens
+ *   cu_seqlens  int32 [num_seqs + 1] device
+ *   B           tokens per block, 1 .. 4096
+ *   keys        uint64 [keys_capacity] device: sequence s's keys at key_cu[s] .. key_cu[s+1]-1
+ *   key_cu      int64 [num_seqs + 1] device: offsets of each sequence's keys
+ * Device-side: offsets outside [0, n] set IAMAP_DEV_BAD_INDEX (the sequence gets no keys); keys
+ * past keys_capacity are not written and set IAMAP_DEV_CAPACITY. Asynchronous on stream.
+ */
+int iamap_prefix_keys(const int32_t* tokens, int64_t n, const int32_t* cu_seqlens, int num_seqs,
+                      int B, uint64_t salt, uint64_t* keys, int64_t keys_capacity,
+                      int64_t* key_cu, void* stream);
+
+/* Empties the table: every key all ones, every location -1. Asynchronous on stream. */
+int iamap_prefix_index_clear(uint64_t* table_keys, int64_t* table_vals, int64_t capacity,
+                             void* stream);
+
+/*
+ * Inserts count (key, location) pairs, keeping the present location of a key that is already
+ * in the table (the first writer wins; among equal keys of one call, one of them). stored
+ * (int64 [count] device) receives, per pair, the location now associated with its key, or -1 for
+ * the reserved empty key and for a pair that found no slot (then IAMAP_DEV_CAPACITY is set).
+ * keys and values are device arrays of count entries. Asynchronous on stream.
+ */
+int iamap_prefix_insert(const uint64_t* keys, const int64_t* values, int64_t count,
+                        uint64_t* table_keys, int64_t* table_vals, int64_t capacity,
+                        int64_t* stored, void* stream);
+
+/*
+ * Looks up count keys: found (int64 [count] device) receives each key's location or -1. With
+ * key_cu (int64 [num_seqs + 1] device, as written by iamap_prefix_keys) and hit_blocks (int32
+ * [num_seqs] device) both non-null, hit_blocks[s] receives the number of leading blocks of
+ * sequence s that were found: its longest cached prefix in blocks. key_cu offsets outside
+ * [0, count] set IAMAP_DEV_BAD_INDEX (that sequence reports 0). Asynchronous on stream.
+ */
+int iamap_prefix_lookup(const uint64_t* keys, int64_t count, const int64_t* key_cu, int num_seqs,
+                        const uint64_t* table_keys, const int64_t* table_vals, int64_t capacity,
+                        int64_t* found, int32_t* hit_blocks, void* stream);
 
 #ifdef __cplusplus
 }

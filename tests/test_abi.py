@@ -103,3 +103,36 @@ def test_host_validation_of_variants(lib):
     assert raw.iamap_mapping_consistency(None, None, 4, None, None) == -1
     assert raw.iamap_selftest_wait_timeout(0, None, None) == -1
     assert raw.iamap_selftest_wait_timeout(2_000_000, None, None) == -1
+
+
+def test_host_validation_of_prefix_index(lib):
+    """The prefix-index entry points refuse bad arguments on the host and count keys there."""
+    raw = lib._lib
+    assert lib.iamap_prefix_num_keys([0, 64, 100, 100, 300], 4, 64) == 4
+    assert lib.iamap_prefix_num_keys([5, 5], 1, 1) == 0
+    n = ctypes.c_int64(0)
+    cu = (ctypes.c_int32 * 3)(0, 10, 4)
+    assert raw.iamap_prefix_num_keys(cu, 2, 4, ctypes.byref(n)) == -1   # decreasing offsets
+    assert raw.iamap_prefix_num_keys(cu, 2, 0, ctypes.byref(n)) == -1   # B < 1
+    fake = 256   # never dereferenced: every call below fails validation first
+    # block size outside [1, 4096]
+    assert raw.iamap_prefix_keys(fake, 64, fake, 1, 0, 0, fake, 1, fake, None) == -1
+    assert raw.iamap_prefix_keys(fake, 64, fake, 1, 4097, 0, fake, 1, fake, None) == -1
+    # null key_cu / null keys with a positive capacity / null tokens with n > 0
+    assert raw.iamap_prefix_keys(fake, 64, fake, 1, 64, 0, fake, 1, None, None) == -1
+    assert raw.iamap_prefix_keys(fake, 64, fake, 1, 64, 0, None, 1, fake, None) == -1
+    assert raw.iamap_prefix_keys(None, 64, fake, 1, 64, 0, fake, 1, fake, None) == -1
+    # capacity not a power of two, or out of range
+    for cap in (0, 3, 100, 1 << 41):
+        assert raw.iamap_prefix_index_clear(fake, fake, cap, None) == -1
+        assert raw.iamap_prefix_insert(fake, fake, 1, fake, fake, cap, fake, None) == -1
+        assert raw.iamap_prefix_lookup(fake, 1, None, 0, fake, fake, cap, fake, None, None) == -1
+    assert "power of two" in lib.iamap_last_error()
+    # null table, null outputs, negative counts, key_cu without hit_blocks
+    assert raw.iamap_prefix_insert(fake, fake, 1, None, fake, 16, fake, None) == -1
+    assert raw.iamap_prefix_insert(fake, fake, 1, fake, fake, 16, None, None) == -1
+    assert raw.iamap_prefix_insert(fake, fake, -1, fake, fake, 16, fake, None) == -1
+    assert raw.iamap_prefix_lookup(fake, 1, fake, 1, fake, fake, 16, fake, None, None) == -1
+    assert "together" in lib.iamap_last_error()
+    assert raw.iamap_prefix_lookup(fake, 1, fake, 0, fake, fake, 16, fake, fake, None) == -1
+    assert raw.iamap_prefix_lookup(None, 1, None, 0, fake, fake, 16, fake, None, None) == -1
