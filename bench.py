@@ -107,14 +107,27 @@ def load_traffic(kernel, workload, files):
 # ------------------------------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clocks and throttle reasons during the timed region (read-only queries).
+
+    nvidia-smi samples every 100 ms; a region shorter than that may get no sample, so an NVML
+    poller (every 2 ms, same GPU index) runs beside it and is used when nvidia-smi took none."""
+
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    # NVML clocks-event reason bits (nvml.h): SwPowerCap 0x4, HwSlowdown 0x8,
+    # SwThermalSlowdown 0x20, HwThermalSlowdown 0x40
+    NVML_BITS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+                 ("hw_thermal_slowdown", 0x40))
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.nvml = []
+        self.nvml_max = 0.0
+        self._poll = None
+        self._halt = threading.Event()
 
     def start(self):
         try:
@@ -130,38 +143,73 @@ class ClockSampler:
             self.lines.clear()   # samples from before the timed region
         except (OSError, FileNotFoundError):
             self.proc = None
+        self._start_nvml()
+
+    def _start_nvml(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.nvml_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception:   # no NVML binding or no device: nvidia-smi alone
+            return
+
+        def poll():
+            while not self._halt.is_set():
+                try:
+                    self.nvml.append((float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                                      int(reasons(h))))
+                except Exception:
+                    return
+                self._halt.wait(0.002)
+
+        self._poll = threading.Thread(target=poll, daemon=True)
+        self._poll.start()
 
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def _stop_nvml(self):
+        if self._poll is not None:
+            self._halt.set()
+            self._poll.join(timeout=2)
+
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.t.join(timeout=2)
+        self._stop_nvml()
         sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 7:
-                continue
+        if self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(parts[0]))
-                mx = max(mx, float(parts[1]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for ln in self.lines:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) < 7:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx = max(mx, float(parts[1]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[3:7]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        if sm:
+            return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                    "reasons": sorted(reasons), "samples": len(sm)}
+        if self.nvml:
+            for _, bits in self.nvml:
+                reasons.update(nm for nm, b in self.NVML_BITS if bits & b)
+            return {"sm_mhz": statistics.median(c for c, _ in self.nvml),
+                    "sm_max_mhz": self.nvml_max, "reasons": sorted(reasons),
+                    "samples": len(self.nvml), "source": "nvml, 2 ms polling"}
+        return None
 
 
 # ------------------------------------------------------------------------------------------------
