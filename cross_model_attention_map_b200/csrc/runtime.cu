@@ -23,8 +23,11 @@ int set_error(int code, const char* fmt, ...) {
 
 void clear_error() { g_last_error[0] = 0; }
 
+// One context per device index, in a fixed array: a context's address never changes, so a
+// pointer returned to one thread stays valid while other threads create other devices' contexts.
+constexpr int kMaxDevices = 64;
 static std::mutex g_ctx_mutex;
-static std::vector<DeviceContext> g_ctx;
+static DeviceContext g_ctx[kMaxDevices];
 
 DeviceContext* device_context() {
   int dev = -1;
@@ -32,8 +35,11 @@ DeviceContext* device_context() {
     set_error(IAMAP_ERR_CUDA, "cudaGetDevice failed");
     return nullptr;
   }
+  if (dev < 0 || dev >= kMaxDevices) {
+    set_error(IAMAP_ERR_UNSUPPORTED, "device index %d beyond %d", dev, kMaxDevices);
+    return nullptr;
+  }
   std::lock_guard<std::mutex> lock(g_ctx_mutex);
-  if ((int)g_ctx.size() <= dev) g_ctx.resize(dev + 1);
   DeviceContext& c = g_ctx[dev];
   if (c.status == nullptr) {
     unsigned int* p = nullptr;
