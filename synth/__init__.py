@@ -22,4 +22,7 @@ from .workloads import (  # noqa: F401
     PrefixWorkload,
     make_prefix_requests,
     prefix_config,
+    ChunkWorkload,
+    chunk_of,
+    make_sender_values,
 )

@@ -316,3 +316,57 @@ def prefix_config(seed: int = 0) -> PrefixWorkload:
     cached set, and 16 prompts of those lengths (four each) looked up against it."""
     lens = [4096, 8192, 12288, 16384]
     return make_prefix_requests(lens, lens * 4, seed=seed)
+
+
+# ----------------------------------------------------------------------------------------------
+# Chunked prefill (a slice of a prefill workload) and sender values
+# ----------------------------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class ChunkWorkload:
+    """Query rows [start, end) of every sequence of a prefill workload, with the keys and values
+    of rows [0, end): the state of a chunked prefill whose earlier chunks are cached."""
+    B: int
+    H_s: int
+    d: int
+    H_r: int
+    d_v: int
+    tau: float
+    bias_window: int
+    bias_value: float
+    W: np.ndarray            # float32 [H_r, H_s]
+    starts: list             # sequence-local first query row of each chunk
+    q: np.ndarray            # uint16 bf16 bits [n_q, H_s, d], chunk rows only
+    cu_q: np.ndarray         # int32 [S+1]
+    k: np.ndarray            # uint16 bf16 bits [n_k, H_s, d], rows [0, end) of every sequence
+    v: np.ndarray            # uint16 bf16 bits [n_k, H_kv, d_v]
+    cu_k: np.ndarray         # int32 [S+1]
+
+
+def chunk_of(wl: PrefillWorkload, starts, ends=None) -> ChunkWorkload:
+    """Slices (no arithmetic): queries of rows [starts[s], ends[s]) and keys/values of rows
+    [0, ends[s]) of sequence s; ends default to the sequence lengths."""
+    ends = list(wl.seqlens) if ends is None else [int(e) for e in ends]
+    qs, ks, vs = [], [], []
+    cu_q, cu_k = [0], [0]
+    for s, (a0, e) in enumerate(zip(starts, ends)):
+        a = int(wl.cu_seqlens[s])
+        if not 0 <= int(a0) <= e <= wl.seqlens[s]:
+            raise ValueError("chunk [%d, %d) outside sequence %d" % (a0, e, s))
+        qs.append(wl.q[a + int(a0):a + e])
+        ks.append(wl.k[a:a + e])
+        vs.append(wl.v[a:a + e])
+        cu_q.append(cu_q[-1] + e - int(a0))
+        cu_k.append(cu_k[-1] + e)
+    return ChunkWorkload(B=wl.B, H_s=wl.H_s, d=wl.d, H_r=wl.H_r, d_v=wl.d_v, tau=wl.tau,
+                         bias_window=wl.bias_window, bias_value=wl.bias_value, W=wl.W,
+                         starts=[int(x) for x in starts], q=np.concatenate(qs),
+                         cu_q=np.array(cu_q, dtype=np.int32), k=np.concatenate(ks),
+                         v=np.concatenate(vs), cu_k=np.array(cu_k, dtype=np.int32))
+
+
+def make_sender_values(wl: PrefillWorkload, d_vs=None, std=1.0, seed=1) -> np.ndarray:
+    """The sender's own values V_s, bf16 bits [n, H_s, d_vs] ~ N(0, std^2), from a generator of
+    their own (so the prefill workload's draws are unchanged)."""
+    rng = np.random.default_rng(seed)
+    return bf16_bits(_normal_bits(rng, (wl.n, wl.H_s, wl.d if d_vs is None else int(d_vs)), std))
