@@ -136,3 +136,57 @@ def test_host_validation_of_prefix_index(lib):
     assert "together" in lib.iamap_last_error()
     assert raw.iamap_prefix_lookup(fake, 1, fake, 0, fake, fake, 16, fake, fake, None) == -1
     assert raw.iamap_prefix_lookup(None, 1, None, 0, fake, fake, 16, fake, None, None) == -1
+
+
+def _prototypes():
+    """name -> number of parameters of every prototype in the header."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(?:int|size_t|const char\s*\*)\s+(iamap_\w+)\s*\(([^)]*)\)\s*;",
+                         text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else len(params.split(","))
+    return out
+
+
+def test_binding_signatures_match_header(lib):
+    """Every ctypes signature of the binding has the header prototype's parameter count, and
+    every header prototype has a signature."""
+    protos = _prototypes()
+    assert len(protos) >= 24
+    sigs = lib._SIGS
+    assert sorted(protos) == sorted(sigs)
+    for name, count in protos.items():
+        assert len(sigs[name][1]) == count, name
+
+
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    """A plain C99 program includes iamap.h, links libiamap.so and calls host-only entry points
+    (planning and argument checks; no device work)."""
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "iamap.h"
+int main(void) {
+  int32_t cu[4] = {0, 64, 100, 300};
+  int64_t rb = 0, cbk = 0, nk = 0;
+  int32_t mx = 0;
+  if (iamap_plan(cu, 3, 64, &rb, &cbk, &mx) != IAMAP_OK) return 1;
+  if (rb != 6 || cbk != 1 + 1 + 10 || mx != 4) return 2;
+  if (iamap_prefix_num_keys(cu, 3, 64, &nk) != IAMAP_OK || nk != 1 + 0 + 3) return 3;
+  if (iamap_prefix_insert(NULL, NULL, 1, NULL, NULL, 3, NULL, NULL) != IAMAP_ERR_INVALID_ARG)
+    return 4;
+  if (iamap_last_error()[0] == 0) return 5;
+  if (iamap_version() < 1) return 6;
+  printf("ok %lld %lld %d %lld\n", (long long)rb, (long long)cbk, mx, (long long)nk);
+  return 0;
+}
+''')
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(lib.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-liamap",
+                    "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
+    assert out.stdout.startswith("ok 6 12 4 4")
