@@ -668,6 +668,44 @@ def oracle_prefix_step(w):
     return (len(w.cached_tokens) + len(w.query_tokens)) / dt, dt
 
 
+def oracle_decode_step(dw):
+    """One float64 oracle decode step (all rows of the batch): (rows/s, seconds)."""
+    import oracle as O
+    t0 = time.perf_counter()
+    O.mapped_av_paged(dw)
+    dt = time.perf_counter() - t0
+    return dw.batch / dt, dt
+
+
+def oracle_headmatch_sample(hm, layers=None):
+    """The float64 oracle calibration on the first `layers` large layers (all of them by default)
+    against every small head: (calibrations/s, seconds). A partial sample counts as
+    layers / L_l of a calibration; the small maps are recomputed in full every time, so that
+    count favours the GPU."""
+    import dataclasses
+    import oracle as O
+    layers = hm.L_l if layers is None else int(layers)
+    sub = dataclasses.replace(hm, L_l=layers, q_large=hm.q_large[:layers],
+                              k_large=hm.k_large[:layers], planted=hm.planted[:layers])
+    t0 = time.perf_counter()
+    O.head_match(sub)
+    dt = time.perf_counter() - t0
+    return (layers / hm.L_l) / dt, dt
+
+
+def _reference_line(args, metric, value, unit, ms, workload, cores_used, sample):
+    print(json.dumps({
+        "impl": "reference", "metric": metric, "value": round(value, 4), "unit": unit,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": workload},
+        "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": cores_used,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }))
+
+
 def reference_arm(args):
     """The float64 oracle on the host cores, same metric and unit, bounded sample per step."""
     from synth import prefill_config
@@ -692,9 +730,32 @@ def reference_arm(args):
                     "d2h_bytes_per_step": 0},
         }))
         return
+    if args.config == "decode":
+        from synth import decode_config
+        dw = decode_config()
+        for _ in range(args.warmup):
+            oracle_decode_step(dw)
+        runs = [oracle_decode_step(dw) for _ in range(args.steps)]
+        value = statistics.mean(v for v, _ in runs)
+        _reference_line(args, "decode rows/s (paged mapped_av, batch 4, context 8704)", value,
+                        "rows/s", 1e3 * dw.batch / value, CONFIG_TEXT["decode"], cores(),
+                        "one whole decode step (batch 4) per step")
+        return
+    if args.config == "headmatch":
+        from synth import head_match_config
+        hm = head_match_config()
+        for _ in range(args.warmup):
+            oracle_headmatch_sample(hm, 1)
+        runs = [oracle_headmatch_sample(hm, 1) for _ in range(args.steps)]
+        value = statistics.mean(v for v, _ in runs)
+        _reference_line(args, "head_match calibrations/s (n=1024, 336 small x 512 large heads)",
+                        value, "calibrations/s", 1e3 / value, CONFIG_TEXT["headmatch"], cores(),
+                        "per step: 1 of the 8 large layers (64 large heads) against all 336 "
+                        "small heads, counted as 1/8 calibration")
+        return
     if args.config not in ("varlen40k", "prefill8k", "tiny"):
         print(json.dumps({"impl": "reference", "unavailable":
-                          "reference arm implemented for the prefill workloads only"}))
+                          "no reference arm for this configuration"}))
         return
     wl = prefill_config(args.config)
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
@@ -754,6 +815,16 @@ def main():
         v, rows, dt, text = oracle_sample_prefill(wl, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(v, 2), "unit": "tokens/s", "cores": cores(),
                                 "kind": "oracle", "sample": text + " in %.1f s" % dt}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "decode":
+        v, dt = oracle_decode_step(wl)
+        line["cpu_baseline"] = {"value": round(v, 3), "unit": "rows/s", "cores": cores(),
+                                "kind": "oracle",
+                                "sample": "one whole decode step (batch 4) in %.1f s" % dt}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "headmatch":
+        v, dt = oracle_headmatch_sample(wl)
+        line["cpu_baseline"] = {"value": round(v, 4), "unit": "calibrations/s",
+                                "cores": cores(), "kind": "oracle",
+                                "sample": "one whole calibration in %.1f s" % dt}
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "prefixindex":
         v, dt = oracle_prefix_step(wl)
         line["cpu_baseline"] = {"value": round(v, 1), "unit": "tokens/s", "cores": 1,

@@ -44,3 +44,25 @@ def test_fewer_than_three_warmup_steps_are_refused():
     r = _run(["--impl", "reference", "--config", "prefixindex", "--steps", "1", "--warmup", "2"])
     assert r.returncode == 2
     assert "warmup" in r.stderr
+
+
+def test_reference_arm_decode_line():
+    r = _run(["--impl", "reference", "--config", "decode", "--steps", "1", "--warmup", "3"])
+    assert r.returncode == 0, r.stderr
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["unit"] == "rows/s" and d["value"] > 0
+    assert d["cpu_baseline"]["cores"] >= 1
+
+
+def test_oracle_timing_helpers_on_small_workloads():
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth import make_decode, make_head_match
+    hm = make_head_match(n=64, L_s=2, H_small=3, d_small=16, L_l=2, H_large=4, d_large=32,
+                         seed=1)
+    full, t_full = bench.oracle_headmatch_sample(hm)
+    half, t_half = bench.oracle_headmatch_sample(hm, 1)
+    assert full > 0 and half > 0 and t_full > 0 and t_half > 0
+    dw = make_decode(batch=2, ctx=100, H_s=3, H_r=4, d_v=16, seed=1)
+    rows, dt = bench.oracle_decode_step(dw)
+    assert abs(rows * dt - 2) < 1e-9
