@@ -347,8 +347,10 @@ int iamap_prefix_insert(const uint64_t* keys, const int64_t* values, int64_t cou
  * Looks up count keys: found (int64 [count] device) receives each key's location or -1. With
  * key_cu (int64 [num_seqs + 1] device, as written by iamap_prefix_keys) and hit_blocks (int32
  * [num_seqs] device) both non-null, hit_blocks[s] receives the number of leading blocks of
- * sequence s that were found: its longest cached prefix in blocks. key_cu offsets outside
- * [0, count] set IAMAP_DEV_BAD_INDEX (that sequence reports 0). Asynchronous on stream.
+ * sequence s that were found: its longest cached prefix in blocks. Then only the keys inside
+ * the sequences' ranges are looked up (all of them when key_cu comes from iamap_prefix_keys).
+ * key_cu offsets outside [0, count] set IAMAP_DEV_BAD_INDEX (that sequence reports 0 and its
+ * found entries are not written). Asynchronous on stream.
  */
 int iamap_prefix_lookup(const uint64_t* keys, int64_t count, const int64_t* key_cu, int num_seqs,
                         const uint64_t* table_keys, const int64_t* table_vals, int64_t capacity,
