@@ -168,7 +168,7 @@ class PrefixIndex:
 
 
 # ------------------------------------------------------------------------------------------------
-# Several GPUs: head matching split by large layers
+# Several GPUs: head matching split by large layers, prefill split by sequence
 # ------------------------------------------------------------------------------------------------
 
 def shard_range(total, world, rank):
@@ -177,6 +177,29 @@ def shard_range(total, world, rank):
     per = -(-total // world)
     lo = min(total, rank * per)
     return lo, min(total, lo + per)
+
+
+def causal_blocks(L, B=64):
+    """Causal (row block, column block) pairs of a sequence of L tokens: its share of the work of
+    compress and mapped_av."""
+    nb = -(-int(L) // B)
+    return nb * (nb + 1) // 2
+
+
+def shard_sequences(seqlens, world, B=64):
+    """Packed sequences -> ranks for a prefill split by sequence (no collective on the path).
+    Longest-processing-time-first: sequences by decreasing causal blocks (ties: lower index)
+    go to the rank with the least work so far (ties: lower rank). The most loaded rank then has
+    at most (4/3 - 1/(3 world)) times the optimum. Returns per-rank lists of sequence indices in
+    increasing order."""
+    work = [0] * world
+    out = [[] for _ in range(world)]
+    order = sorted(range(len(seqlens)), key=lambda s: (-causal_blocks(seqlens[s], B), s))
+    for s in order:
+        r = min(range(world), key=lambda x: (work[x], x))
+        out[r].append(s)
+        work[r] += causal_blocks(seqlens[s], B)
+    return [sorted(x) for x in out]
 
 
 def gather_head_mapping(local_argmax, L_l, H_large, group=None):

@@ -25,4 +25,5 @@ from .workloads import (  # noqa: F401
     ChunkWorkload,
     chunk_of,
     make_sender_values,
+    select_sequences,
 )

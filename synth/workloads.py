@@ -370,3 +370,15 @@ def make_sender_values(wl: PrefillWorkload, d_vs=None, std=1.0, seed=1) -> np.nd
     their own (so the prefill workload's draws are unchanged)."""
     rng = np.random.default_rng(seed)
     return bf16_bits(_normal_bits(rng, (wl.n, wl.H_s, wl.d if d_vs is None else int(d_vs)), std))
+
+
+def select_sequences(wl: PrefillWorkload, idx) -> PrefillWorkload:
+    """The packed workload of sequences `idx` of `wl` (in that order): slices, no arithmetic."""
+    idx = [int(s) for s in idx]
+    parts = [slice(int(wl.cu_seqlens[s]), int(wl.cu_seqlens[s + 1])) for s in idx]
+    lens = [wl.seqlens[s] for s in idx]
+    cu = np.zeros(len(idx) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lens) if lens else []
+    cat = (lambda a: np.concatenate([a[p] for p in parts]) if parts else a[:0])
+    return dataclasses.replace(wl, seqlens=lens, q=cat(wl.q), k=cat(wl.k), v=cat(wl.v),
+                               cu_seqlens=cu)

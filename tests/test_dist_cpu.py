@@ -95,3 +95,54 @@ def test_sharded_head_match_equals_single_process():
     _, ref = O.head_match(hm)
     for rank in (0, 1):
         np.testing.assert_array_equal(np.array(out[rank]), ref)
+
+
+def _brute_makespan(work, world):
+    best = None
+    for assign in np.ndindex(*([world] * len(work))):
+        loads = [0] * world
+        for w, r in zip(work, assign):
+            loads[r] += w
+        best = max(loads) if best is None else min(best, max(loads))
+    return best
+
+
+def test_shard_sequences_balances_causal_work():
+    """Every sequence goes to exactly one rank, and the most loaded rank is within the
+    longest-first bound of the optimum found by brute force."""
+    from cross_model_attention_map_b200.runner import causal_blocks, shard_sequences
+    rng = np.random.default_rng(3)
+    for trial in range(40):
+        lens = [int(x) for x in rng.integers(0, 700, size=int(rng.integers(1, 8)))]
+        for world in (1, 2, 3):
+            parts = shard_sequences(lens, world, B=64)
+            assert sorted(s for p in parts for s in p) == list(range(len(lens)))
+            work = [causal_blocks(L, 64) for L in lens]
+            got = max(sum(work[s] for s in p) for p in parts)
+            opt = _brute_makespan(work, world)
+            assert got * 3 * world <= opt * (4 * world - 1)
+    # the varlen packing (4096/8192/12288/16384) on 2 ranks: 16384 alone against the rest
+    assert shard_sequences([4096, 8192, 12288, 16384], 2) == [[3], [0, 1, 2]]
+
+
+def test_prefill_split_by_sequence_equals_whole_batch():
+    """Each rank's share of the packed sequences, run on its own, gives exactly the rows of the
+    whole batch (the oracle stands in for each rank's GPU step; there is no exchange)."""
+    import oracle as O
+    from synth import make_prefill, select_sequences
+    from cross_model_attention_map_b200.runner import shard_sequences
+    wl = make_prefill([90, 30, 150, 64, 7], H_s=2, d=16, H_r=3, d_v=8, B=16, tau=0.8, seed=12)
+    res = O.compress(wl)
+    whole = O.mapped_av(wl, res.kept)
+    for world in (2, 3):
+        for part in shard_sequences(wl.seqlens, world, B=16):
+            if not part:
+                continue
+            sub = select_sequences(wl, part)
+            r = O.compress(sub)
+            o = O.mapped_av(sub, r.kept)
+            for i, s in enumerate(part):
+                a, b = int(wl.cu_seqlens[s]), int(wl.cu_seqlens[s + 1])
+                c = int(sub.cu_seqlens[i])
+                np.testing.assert_array_equal(o[c:c + b - a], whole[a:b])
+                np.testing.assert_array_equal(r.lse[:, c:c + b - a], res.lse[:, a:b])
