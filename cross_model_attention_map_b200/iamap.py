@@ -72,6 +72,8 @@ _SIGS = {
     "iamap_mapping_consistency": (_I, [_P, _P, _I, _P, _P]),
     "iamap_selftest_wait_timeout": (_I, [_I, _P, _P]),
     "iamap_prefix_num_keys": (_I, [_P, _I, _I, ctypes.POINTER(_I64)]),
+    "iamap_bsr_check_host": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I64,
+                                  ctypes.POINTER(_I64)]),
     "iamap_prefix_keys": (_I, [_P, _I64, _P, _I, _I, _U64, _P, _I64, _P, _P]),
     "iamap_prefix_index_clear": (_I, [_P, _P, _I64, _P]),
     "iamap_prefix_insert": (_I, [_P, _P, _I64, _P, _P, _I64, _P, _P]),
@@ -275,6 +277,22 @@ def iamap_head_match(q_small, k_small, L_s, H_small, d_small, q_large, k_large, 
         _ptr(q_small), _ptr(k_small), L_s, H_small, d_small, _ptr(q_large), _ptr(k_large), L_l,
         H_large, d_large, n, n_used, _ptr(argmax), _ptr(sim), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def iamap_bsr_check_host(cu_seqlens_host, num_seqs, B, H_s, row_ptr, col_idx, headmask, val_off,
+                         vals_capacity_tiles):
+    """Host structure check of a block-sparse map (host arrays or CPU tensors). Returns
+    (status, first offending block or -1, message); does not raise on an invalid map."""
+    def host(a, dtype):
+        t = torch.as_tensor(a).cpu().contiguous()
+        return t.view(dtype) if t.dtype.itemsize == dtype.itemsize else t.to(dtype)
+    cu, _k0 = _host_i32(cu_seqlens_host)
+    rp, ci = host(row_ptr, torch.int32), host(col_idx, torch.int32)
+    hm, vo = host(headmask, torch.int64), host(val_off, torch.int64)
+    bad = _I64(-1)
+    rc = _lib.iamap_bsr_check_host(cu, num_seqs, B, H_s, _ptr(rp), _ptr(ci), _ptr(hm), _ptr(vo),
+                                   vals_capacity_tiles, ctypes.byref(bad))
+    return rc, bad.value, iamap_last_error()
 
 
 def iamap_prefix_num_keys(cu_seqlens_host, num_seqs, B) -> int:

@@ -286,6 +286,22 @@ int iamap_head_match_metric(const void* q_small, const void* k_small, int L_s, i
 int iamap_mapping_consistency(const int32_t* a, const int32_t* b, int n_heads, int32_t* agree,
                               void* stream);
 
+/*
+ * Structure check of a block-sparse map on the host (e.g. one read back from storage or from
+ * another process before mapped_av uses it). All pointers are HOST pointers; nothing is written
+ * except *bad_block. The map is valid when, for every row block I of every sequence:
+ * row_ptr starts at 0 and does not decrease; the column blocks of a row block ascend strictly
+ * and lie in 0..I; each head mask is non-zero with bits only below H_s; and each block's tiles
+ * [val_off, val_off + popcount(mask)) lie in [0, vals_capacity_tiles).
+ * Returns IAMAP_OK, IAMAP_ERR_INVALID_ARG (bad structure or arguments) or IAMAP_ERR_CAPACITY
+ * (tiles outside the buffer); *bad_block (if non-null) receives the first offending block, or
+ * -1. iamap_last_error names the violation.
+ */
+int iamap_bsr_check_host(const int32_t* cu_seqlens_host, int num_seqs, int B, int H_s,
+                         const int32_t* row_ptr, const int32_t* col_idx, const uint64_t* headmask,
+                         const int64_t* val_off, int64_t vals_capacity_tiles,
+                         int64_t* bad_block);
+
 /* ---------------------------------------------------------------------------------------------
  * Prefix-hash block index ("PKU MapFlow: cross-model attention map reuse" news page, storage-
  * and-execution part, second component: stored map blocks are located through a prefix hash
