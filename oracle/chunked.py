@@ -16,7 +16,7 @@ Sources:
 [MapFlow-maps]  same page, the attention map as the shared state: the sender runs its own
                 attention; the receiver reuses the sender's probabilities with its own V.
 
-Readings (each also listed in the design doc):
+Readings where the pages are silent:
 
 * a chunk of sequence s is its query rows [c0, e); it attends to keys [0, e) with the same
   causal mask and bias as the whole sequence (absolute positions). c0 is a multiple of B, so the

@@ -32,7 +32,7 @@ Sources (cited below by the short tag in brackets):
                model's attention directly (no Q/K projection, no QK^T, no K cache); prompts longer
                than tau_t are truncated for the similarity computation.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 * cumulative-mass selection is per (sender head, row block) and normalised by the row block's
   total mass, which equals its number of valid rows; tau >= 1 keeps every causal block;
 * ties between equal block masses are broken by the lower column-block index;

@@ -15,8 +15,7 @@ Source:
               basis 0xcbf29ce484222325, and each octet is XORed into the state, which is then
               multiplied by the prime 0x100000001b3 modulo 2**64.
 
-The page fixes no hash function, block size or table layout. The readings used here (each also
-listed in DESIGN.md):
+The page fixes no hash function, block size or table layout. The readings used here:
 
 * blocks are the map's row blocks: B consecutive tokens of one packed sequence, starting at a
   multiple of B; only full blocks are indexed, because a partial last block changes once the
