@@ -58,6 +58,24 @@ def test_keys_parity_ragged_small_blocks(lib):
     assert status(C) == 0
 
 
+def test_keys_parity_prompts_longer_than_one_chunk(lib):
+    """Prompts of 312 and 257 blocks: the keys kernel digests 256 blocks per pass and carries the
+    chain state from one pass to the next."""
+    C, runner = lib
+    rng = np.random.default_rng(2)
+    lens = [5000, 17, 0, 4113, 300]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    toks = rng.integers(-2**31, 2**31 - 1, size=int(cu[-1]), dtype=np.int64).astype(np.int32)
+    salt = 0x1234567890ABCDEF
+    idx = runner.PrefixIndex(64, B=16, salt=salt)
+    keys, key_cu = gpu_keys(runner, idx, toks, cu)
+    ref, ref_cu = px.prefix_keys(toks, cu, 16, salt)
+    assert list(np.diff(ref_cu)) == [312, 1, 0, 257, 18]
+    assert np.array_equal(key_cu.cpu().numpy(), ref_cu)
+    assert np.array_equal(keys_np(keys), ref)
+    assert status(C) == 0
+
+
 def test_keys_parity_full_size_prompts(lib):
     """The varlen prompt set (4 cached prompts of 4096..16384 tokens, 16 prompts looked up),
     B = 64: every key bit-exact."""
