@@ -176,6 +176,11 @@ class ClockSampler:
         if self._poll is not None:
             self._halt.set()
             self._poll.join(timeout=2)
+            try:
+                import pynvml
+                pynvml.nvmlShutdown()
+            except Exception:
+                pass
 
     def stop(self):
         self._stop_nvml()
