@@ -11,13 +11,20 @@
 // even the status word the other entry points create on first use.
 //
 // Limits and behaviour:
-//   * The scratch array holds kNoAllocScratchFloats floats (16 MiB). Every GPU that loads the
-//     library holds that much device memory until the process exits. A call whose split partial
-//     sums (batch x chunks x H_r x d_v floats, chunks chosen as in iamap_mapped_av_paged) do not fit
-//     returns IAMAP_ERR_CAPACITY without launching anything.
-//   * On the first call on a device, with that device current, the call looks up the device
-//     address of the array (cudaGetSymbolAddress) and caches it; later calls on that device reuse
-//     it. Make that first call before any stream capture.
+//   * The scratch array holds kNoAllocScratchFloats floats (16 MiB). It belongs to this file's
+//     device module. With CUDA's lazy module loading (the default) the module, and with it the
+//     16 MiB of device memory, is loaded by the first call on each device (the address look-up
+//     below), not when the library is loaded; the decode kernels' own module likewise loads on
+//     its first launch. So the FIRST call on a device does take device memory, and may
+//     synchronise. Make that first call at start-up, before reserving the rest of the GPU's memory
+//     and before any stream capture; from then on the device holds the array until the process
+//     exits, and calls allocate nothing.
+//   * A call whose split partial sums (batch x chunks x H_r x d_v floats, chunks chosen as in
+//     iamap_mapped_av_paged) do not fit returns IAMAP_ERR_CAPACITY without launching anything.
+//   * The device address of the array is looked up with cudaGetSymbolAddress, with the device
+//     current, and cached per (device, current context). A call from another context on the same
+//     device (a driver-API context, or the primary context re-created after cudaDeviceReset)
+//     looks it up again, so a stale address is never used.
 //   * All calls on a device share the one array, and it keeps the previous call's contents. The
 //     kernel writes every partial sum it later reads, so nothing needs clearing between calls, but
 //     two calls whose work overlaps on the GPU (different streams, no ordering between them) race
@@ -38,24 +45,55 @@ constexpr int kNoAllocMaxDevices = 64;
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
 static std::mutex g_noalloc_mutex;
-static float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+struct NoAllocSlot {
+  void* ctx = nullptr;    // the context the address was looked up in
+  float* ptr = nullptr;
+};
+static NoAllocSlot g_noalloc_slot[kNoAllocMaxDevices];
 
-// Device address of the scratch array on the current device (looked up once per device).
+// The current context of the calling thread (cuCtxGetCurrent through the runtime's driver entry
+// point, so the library needs no libcuda link).
+static int current_context(void** ctx) {
+  using GetCurrent = int (*)(void**);
+  static GetCurrent fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetCurrent>(f);
+  });
+  if (!fn) return set_error(IAMAP_ERR_CUDA, "cuCtxGetCurrent is unavailable");
+  if (fn(ctx) != 0) return set_error(IAMAP_ERR_CUDA, "cuCtxGetCurrent failed");
+  return IAMAP_OK;
+}
+
+// Device address of the scratch array in the current context of the current device (looked up
+// once per device and context).
 static int noalloc_scratch(float** out) {
   int dev = -1;
   IAMAP_CUDA_CHECK(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kNoAllocMaxDevices)
     return set_error(IAMAP_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kNoAllocMaxDevices);
+  void* ctx = nullptr;
+  int rc = current_context(&ctx);
+  if (rc) return rc;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  NoAllocSlot& slot = g_noalloc_slot[dev];
+  if (ctx == nullptr || slot.ptr == nullptr || slot.ctx != ctx) {
+    // (a thread with no current context gets the device's primary context from the look-up)
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr)
       return set_error(IAMAP_ERR_CUDA, "cudaGetSymbolAddress of the decode scratch failed: %s",
                        cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = static_cast<float*>(p);
+    rc = current_context(&ctx);
+    if (rc) return rc;
+    slot.ctx = ctx;
+    slot.ptr = static_cast<float*>(p);
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return IAMAP_OK;
 }
 

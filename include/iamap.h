@@ -224,11 +224,15 @@ int iamap_mapped_av_paged_gqa(const float* p_rows, int ctx_stride, const float* 
  * cache at start-up, or one that forbids cudaMalloc on its decode loop because cudaMalloc
  * synchronises the device. The pages have no counterpart of this entry point; it exists only
  * for such callers. Same arguments and result as iamap_mapped_av_paged, minus the workspace:
- * the split partial sums live in a fixed 16 MiB device array inside the library, which every GPU
- * that loads the library holds until the process exits. Nothing here allocates (no cudaMalloc,
- * no cudaFree, no status word).
- *   - The first call on a device looks up that array's device address and caches it; make that
- *     first call before any stream capture.
+ * the split partial sums live in a fixed 16 MiB device array inside the library. The call itself
+ * allocates nothing (no cudaMalloc, no cudaFree, no status word), with one exception:
+ *   - Under CUDA's lazy module loading (the default) the array, and the decode kernels, are
+ *     loaded onto a device by the FIRST call on that device, which therefore takes 16 MiB of
+ *     device memory (plus the kernels' code) and may synchronise. Make that first call at
+ *     start-up, before reserving the rest of the GPU's memory and before any stream capture;
+ *     the device then holds the array until the process exits.
+ *   - The array's device address is looked up (cudaGetSymbolAddress) per device and current
+ *     context, so a call from another context, or after cudaDeviceReset, looks it up again.
  *   - A call whose partial sums (batch x chunks x H_r x d_v floats) exceed 16 MiB returns
  *     IAMAP_ERR_CAPACITY and launches nothing.
  *   - All calls on a device share the array (it keeps the last call's contents; every value read

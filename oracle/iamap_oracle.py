@@ -153,10 +153,16 @@ def select_blocks(masses: np.ndarray, R: int, tau: float, eps: float = NEAR_EPS)
     cumulative mass reaches tau * R. tau >= 1 keeps all blocks.
 
     Returns (kept, near): boolean arrays over J. ``near`` marks blocks whose membership could flip
-    under a perturbation of the normalised masses by eps: a block whose normalised mass is within
-    eps of the last kept block's, the last kept block when the cumulative mass before it is within
-    eps of tau, and the first dropped block when the cumulative mass through the last kept one is
-    within eps of tau.
+    under a perturbation of the normalised masses by eps. The selection threshold is the
+    normalised mass t of the last kept block; three cases can flip:
+      (a) a dropped block whose normalised mass is within eps of t: it can change places with the
+          last kept block, so it, the last kept block and any other block within eps of t are
+          near (the last kept block is never compared with its own mass: clear margins mark
+          nothing);
+      (b) the cumulative mass before the last kept block is within eps of tau: that block may not
+          be needed, and neither may any kept block within eps of t that could take its place;
+      (c) the cumulative mass through the last kept block is within eps of tau: the first dropped
+          block may be needed, and so may any dropped block within eps of its mass.
     """
     nJ = len(masses)
     kept = np.zeros(nJ, dtype=bool)
@@ -177,12 +183,18 @@ def select_blocks(masses: np.ndarray, R: int, tau: float, eps: float = NEAR_EPS)
         cum_before_last = cum
         cum += mhat[J]
         cum_through_last = cum
-    thr = mhat[order[last]]
-    near |= np.abs(mhat - thr) <= eps
-    if abs(cum_before_last - tau) <= eps:
-        near[order[last]] = True
-    if last + 1 < nJ and abs(cum_through_last - tau) <= eps:
-        near[order[last + 1]] = True
+    if last < 0:
+        return kept, near
+    J_last = order[last]
+    close_t = np.abs(mhat - mhat[J_last]) <= eps
+    if (close_t & ~kept).any():                                       # (a)
+        near |= close_t
+    if abs(cum_before_last - tau) <= eps:                             # (b)
+        near |= close_t & kept
+        near[J_last] = True
+    if last + 1 < nJ and abs(cum_through_last - tau) <= eps:          # (c)
+        J_first = order[last + 1]
+        near |= (np.abs(mhat - mhat[J_first]) <= eps) & ~kept
     return kept, near
 
 

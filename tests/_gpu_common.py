@@ -3,6 +3,8 @@ and the comparison rules (tolerances of the benchmark description)."""
 
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -43,13 +45,34 @@ def check_output(o_gpu: np.ndarray, o_ref: np.ndarray, what=""):
     return rel, mx
 
 
-def compare_kept(kept_gpu: np.ndarray, kept_ref: np.ndarray, near: np.ndarray):
-    """Bit-exact outside near-threshold blocks; returns the number of (near-threshold) flips."""
+def compare_kept(kept_gpu: np.ndarray, kept_ref: np.ndarray, near: np.ndarray, report=True):
+    """Bit-exact outside near-threshold blocks; returns the number of (near-threshold) flips.
+    The counts of compared, near and flipped blocks go to the end-of-run report."""
     diff = kept_gpu != kept_ref
     bad = diff & ~near
     assert not bad.any(), "kept sets differ outside near-threshold blocks at %s" % (
         list(zip(*np.nonzero(bad)))[:10],)
-    return int(diff.sum())
+    flips = int(diff.sum())
+    if report:
+        import conftest
+        name = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+        conftest.KEPT_REPORT.append((name, int(kept_ref.size), int(near.sum()), flips))
+    return flips
+
+
+def check_kept_invariants(kept, mass_norm, tau, eps=1e-5):
+    """The cumulative-mass choice of every (head, row block), checked on a kept set with the
+    given normalised masses [H, blocks of the row block]: the kept mass reaches tau, dropping the
+    smallest kept block falls below it, and no dropped block outweighs a kept one."""
+    if tau >= 1.0:
+        assert kept.all()
+        return
+    km = (mass_norm * kept).sum(axis=1)
+    assert (km >= tau - eps).all(), "kept mass below tau: %s" % (km.min(),)
+    mn = np.where(kept, mass_norm, np.inf).min(axis=1)
+    assert (km - mn < tau + eps).all(), "kept set is not minimal"
+    mx = np.where(~kept, mass_norm, -np.inf).max(axis=1)
+    assert (mx <= mn + eps).all(), "a dropped block outweighs a kept one"
 
 
 def bsr_readback(layer):

@@ -16,3 +16,17 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def root():
     return ROOT
+
+
+# Near-threshold report: every kept-set comparison records how many blocks the oracle marked
+# near the selection threshold and how many of them the GPU decided the other way; the counts are
+# printed at the end of the run.
+KEPT_REPORT = []
+
+
+def pytest_terminal_summary(terminalreporter):
+    if not KEPT_REPORT:
+        return
+    terminalreporter.section("kept-set comparisons (near-threshold blocks, flips)")
+    for name, blocks, near, flips in KEPT_REPORT:
+        terminalreporter.write_line("%-70s blocks %8d  near %4d  flips %4d" % (name, blocks, near, flips))

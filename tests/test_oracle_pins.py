@@ -183,6 +183,93 @@ def test_brute_force_selection_small():
 
 
 # ----------------------------------------------------------------------------------------------
+# Near-threshold blocks on hand-built mass vectors (the tolerance of the kept-set comparison)
+# ----------------------------------------------------------------------------------------------
+
+# Each case: normalised masses, tau, the kept set and the near set worked out by hand. R = 64
+# rows, so the masses passed are 64 times these.
+_NEAR_CASES = [
+    # clear margins everywhere: nothing is near (the last kept block, J=2, is not compared with
+    # its own mass)
+    ("clear", [0.5, 0.3, 0.15, 0.05], 0.9, {0, 1, 2}, set()),
+    # the last kept block (J=2) and a dropped block (J=3) have equal masses: the order between
+    # them may swap, both are near
+    ("equal", [0.5, 0.3, 0.1, 0.1], 0.85, {0, 1, 2}, {2, 3}),
+    # a dropped block 4e-6 below the last kept one: both near
+    ("close", [0.5, 0.3, 0.1, 0.1 - 4e-6], 0.85, {0, 1, 2}, {2, 3}),
+    # a dropped block 3e-5 below the last kept one: a clear margin
+    ("apart", [0.5, 0.3, 0.1, 0.1 - 3e-5], 0.85, {0, 1, 2}, set()),
+    # the cumulative mass before the last kept block (J=2) lands 5e-6 below tau: J=2 is near
+    ("cum_before", [0.6, 0.3 - 5e-6, 0.08 + 5e-6, 0.02], 0.9, {0, 1, 2}, {2}),
+    # the cumulative mass through the last kept block (J=1) lands 5e-6 above tau: the first
+    # dropped block (J=2) is near
+    ("cum_through", [0.6, 0.3 + 5e-6, 0.08, 0.02 - 5e-6], 0.9, {0, 1}, {2}),
+    # ties in the order: equal masses sort by lower J, so J=1 is kept before J=3; the last kept
+    # block is J=3 and no other block is close to its mass
+    ("tie_order", [0.1, 0.3, 0.55, 0.3, 0.0], 0.9, {1, 2, 3}, set()),
+]
+
+
+@pytest.mark.parametrize("name,mh,tau,kept_exp,near_exp", _NEAR_CASES, ids=[c[0] for c in _NEAR_CASES])
+def test_near_threshold_hand_built(name, mh, tau, kept_exp, near_exp):
+    R = 64
+    kept, near = O.select_blocks(np.array(mh) * R, R, tau)
+    assert set(np.flatnonzero(kept)) == kept_exp
+    assert set(np.flatnonzero(near)) == near_exp
+
+
+def test_near_threshold_is_rare_on_the_tiny_workload():
+    """With the rule above, near-threshold blocks are the exception: on the tiny configuration
+    (8 heads x 36 causal blocks) no block is near, and in particular no last kept block is."""
+    from synth import prefill_config
+    wl = prefill_config("tiny")
+    res = O.compress(wl)
+    assert res.near.sum() <= 2, int(res.near.sum())
+
+
+def test_dropping_the_last_kept_block_is_caught():
+    """A planted selection mistake (the oracle's own kept sets with the last kept block of one
+    row block removed) fails the kept-set comparison the GPU tests use."""
+    from _gpu_common import compare_kept
+    wl = make_prefill([300], H_s=3, d=32, H_r=2, d_v=8, B=32, tau=0.9, std=1.5, sink=True, seed=6)
+    res = O.compress(wl)
+    lay = res.layout
+    assert compare_kept(res.kept, res.kept, res.near, report=False) == 0
+    I = 7
+    st = O.rowblock_stats(wl.q, wl.k, wl.cu_seqlens, 0, 1, I, wl.B, wl.tau)
+    mh = st.masses / st.R
+    kept_J = np.flatnonzero(st.kept)
+    last = kept_J[np.argmin(mh[kept_J] + 1e-12 * kept_J)]   # smallest kept mass (ties: higher J)
+    assert not res.near[1, lay.cb(0, I, last)]
+    bad = res.kept.copy()
+    bad[1, lay.cb(0, I, last)] = False
+    with pytest.raises(AssertionError):
+        compare_kept(bad, res.kept, res.near, report=False)
+
+
+# ----------------------------------------------------------------------------------------------
+# Closed form: Q = 0 gives uniform rows p_ij = 1/(i+1)
+# ----------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("L,I,J", [(100, 1, 1), (100, 1, 0), (64, 0, 0), (70, 1, 1)])
+def test_masked_tile_partial_blocks_closed_form(L, I, J):
+    """masked_tile on uniform rows (Q = 0): entry (r, c) of the tile of column block J in row
+    block I is 1/(i+1) for the global row i = 64 I + r and column j = 64 J + c when i < L and
+    j <= i, and 0 otherwise (exact rationals; partial last blocks of a sequence of L tokens)."""
+    B = 64
+    wl = make_prefill([L], H_s=1, d=16, H_r=1, d_v=4, B=B, tau=1.0, q_zero=True, seed=3)
+    st = O.rowblock_stats(wl.q, wl.k, wl.cu_seqlens, 0, 0, I, B, 1.0)
+    t = O.masked_tile(st, J, B)
+    assert t.shape == (B, B)
+    for r in range(B):
+        i = I * B + r
+        for c in range(B):
+            j = J * B + c
+            exp = Fraction(1, i + 1) if (i < L and j <= i) else Fraction(0)
+            assert abs(t[r, c] - float(exp)) < 1e-15, (r, c)
+
+
+# ----------------------------------------------------------------------------------------------
 # Closed form: Q = 0 gives uniform rows p_ij = 1/(i+1)
 # ----------------------------------------------------------------------------------------------
 
