@@ -420,9 +420,9 @@ def bench_prefill(args, world, rank, local, peaks):
                 "peak_source": peaks["source"] + {"TFLOP/s": " sustained bf16", "GB/s": " HBM copy",
                                                    "Gex2/s": " (16 ex2/clk/SM x 148 SMs x max clock)"}[unit]}
 
-    # end to end through the public API with host buffers (pinned): every step uploads its q, k,
-    # v, W and reads its output back; HostPrefillPipeline overlaps the next step's upload and the
-    # previous step's read-back with the current step's kernels.
+    # end to end through the library's host-buffer entry point (iamap_prefill_steps_host, pinned
+    # host buffers): every step uploads its q, k, v, W and reads its output back; the next step's
+    # upload and the previous step's read-back overlap the current step's kernels.
     from cross_model_attention_map_b200.runner import HostPrefillPipeline
     hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True); hq.copy_(q)
     hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True); hk.copy_(k)
@@ -439,7 +439,7 @@ def bench_prefill(args, world, rank, local, peaks):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    e1 = pipe.run(ins, outs, stream, start_event=e0)
+    e1 = pipe.run(ins, outs, stream)
     torch.cuda.synchronize()
     h2d, d2h = pipe.bytes_per_step()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)

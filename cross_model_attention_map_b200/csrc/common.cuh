@@ -51,7 +51,22 @@ struct SeqTables {
   int64_t* row_tiles; // [num_rowblocks] tiles of each row block (then their exclusive scan)
   int2* pairs;        // [num_pairs] (seq, I0) of the row-block pairs (I0, I0 + 1), I0 even,
                       // longest first
+  // Chunked prefill: sequence s contributes only its row blocks I >= I0[s] (its query rows
+  // [B * I0[s], L_s)), and the query (and output) row of sequence-local row i is packed at
+  // qoff[s] + i. Whole sequences have I0 = 0 and qoff = cu_seqlens[s].
+  int32_t* I0;        // [num_seqs]
+  int32_t* qoff;      // [num_seqs]
 };
+
+// Index of row block I of sequence s among the row blocks listed in the tables.
+__device__ __forceinline__ int tab_rb(const SeqTables& t, int s, int I) {
+  return t.rb_start[s] + I - t.I0[s];
+}
+// Index of causal block (I, 0) of sequence s among the causal blocks listed in the tables.
+__device__ __forceinline__ int64_t tab_cb(const SeqTables& t, int s, int I) {
+  const int64_t i0 = t.I0[s];
+  return (int64_t)t.cb_start[s] + (int64_t)I * (I + 1) / 2 - i0 * (i0 + 1) / 2;
+}
 size_t seq_tables_bytes(int num_seqs, int64_t num_rowblocks);
 SeqTables carve_seq_tables(void* ws, int num_seqs, int64_t num_rowblocks);
 
@@ -63,10 +78,18 @@ struct Plan {
   int64_t num_pairs = 0;   // sum over sequences of ceil(nb / 2)
 };
 int make_plan(const int32_t* cu_host, int num_seqs, int B, int64_t n, Plan* out);
+// Plan of the chunks of packed sequences: sequence s has keys [0, cu_k[s+1] - cu_k[s]) and query
+// rows [starts[s], that length), starts[s] a multiple of B; the query rows are packed by
+// cu_q (cu_q[s+1] - cu_q[s] rows each, n_q in all). Only the chunk's row blocks are counted.
+int make_chunk_plan(const int32_t* cu_k_host, const int32_t* cu_q_host,
+                    const int32_t* starts_host, int num_seqs, int B, int64_t n_k, int64_t n_q,
+                    Plan* out);
 
-// Builds SeqTables on the device from cu_seqlens (device), on `stream`.
+// Builds SeqTables on the device from cu_seqlens (device), on `stream`. With cu_q and starts
+// (device, both non-null) the tables list only each sequence's chunk (see make_chunk_plan).
 int launch_build_tables(const int32_t* cu_seqlens, int num_seqs, int B, int32_t max_nb,
-                        SeqTables t, cudaStream_t stream);
+                        SeqTables t, cudaStream_t stream, const int32_t* cu_q = nullptr,
+                        const int32_t* starts = nullptr);
 
 // ------------------------------------------------------------------------------------------------
 // Device side helpers

@@ -114,8 +114,8 @@ __global__ void __launch_bounds__(kTileThreads) compress_kernel(CompressParams p
   const int64_t rs = (int64_t)p.H_s * D;
   const __nv_bfloat16* qb = p.q + (int64_t)seq0 * rs + (int64_t)h * D;
   const __nv_bfloat16* kb = p.k + (int64_t)seq0 * rs + (int64_t)h * D;
-  const int rb = p.tab.rb_start[s] + I;
-  const int cb0 = p.tab.cb_start[s] + I * (I + 1) / 2;
+  const int rb = tab_rb(p.tab, s, I);
+  const int64_t cb0 = tab_cb(p.tab, s, I);
 
   const uint32_t sK0 = smem_u32(smem);
   constexpr uint32_t kStage = kTile * D * 2;
@@ -303,8 +303,8 @@ __global__ void row_count_kernel(const unsigned long long* __restrict__ hm_dense
   const int lane = threadIdx.x & 31;
   if (item >= num_rowblocks) return;
   const int2 it = tab.items[item];
-  const int rb = tab.rb_start[it.x] + it.y;
-  const int cb0 = tab.cb_start[it.x] + it.y * (it.y + 1) / 2;
+  const int rb = tab_rb(tab, it.x, it.y);
+  const int64_t cb0 = tab_cb(tab, it.x, it.y);
   int cnt = 0;
   long long tiles = 0;
   for (int J = lane; J <= it.y; J += 32) {
@@ -381,8 +381,8 @@ __global__ void row_fill_kernel(const unsigned long long* __restrict__ hm_dense,
   const int lane = threadIdx.x & 31;
   if (item >= num_rowblocks) return;
   const int2 it = tab.items[item];
-  const int rb = tab.rb_start[it.x] + it.y;
-  const int cb0 = tab.cb_start[it.x] + it.y * (it.y + 1) / 2;
+  const int rb = tab_rb(tab, it.x, it.y);
+  const int64_t cb0 = tab_cb(tab, it.x, it.y);
   int u = row_ptr[rb];
   long long toff = tab.row_tiles[rb];
   for (int base = 0; base <= it.y; base += 32) {
@@ -462,14 +462,19 @@ int compress_stats_impl(const CompressArgs& a, cudaStream_t stream) {
   if (rc) return rc;
   const int64_t nrb = a.plan.num_rowblocks;
   const unsigned wgrid = (unsigned)((nrb * 32 + 255) / 256);
-  row_count_kernel<<<wgrid, 256, 0, stream>>>(p.headmask_dense, a.tab, nrb, a.row_ptr);
-  IAMAP_LAUNCH_CHECK("row_count_kernel");
+  if (wgrid > 0) {
+    row_count_kernel<<<wgrid, 256, 0, stream>>>(p.headmask_dense, a.tab, nrb, a.row_ptr);
+    IAMAP_LAUNCH_CHECK("row_count_kernel");
+  }
+  // (with no row blocks this writes row_ptr[0] = 0 and zero counts)
   row_scan_kernel<<<1, 1024, 0, stream>>>(a.row_ptr, a.tab.row_tiles, nrb, a.counts);
   IAMAP_LAUNCH_CHECK("row_scan_kernel");
-  row_fill_kernel<<<wgrid, 256, 0, stream>>>(p.headmask_dense, a.tab, nrb, a.row_ptr, a.col_idx,
-                                             reinterpret_cast<unsigned long long*>(a.headmask),
-                                             a.val_off);
-  IAMAP_LAUNCH_CHECK("row_fill_kernel");
+  if (wgrid > 0) {
+    row_fill_kernel<<<wgrid, 256, 0, stream>>>(p.headmask_dense, a.tab, nrb, a.row_ptr, a.col_idx,
+                                               reinterpret_cast<unsigned long long*>(a.headmask),
+                                               a.val_off);
+    IAMAP_LAUNCH_CHECK("row_fill_kernel");
+  }
   return IAMAP_OK;
 }
 

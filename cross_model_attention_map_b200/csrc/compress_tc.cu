@@ -45,6 +45,13 @@ enum { Q_FULL = 0, K_FULL = 1, K_EMPTY = K_FULL + kSStages, S_FULL = K_EMPTY + k
 constexpr int kXBufs = 4;          // extract: S buffers of 64 TMEM columns (two per writer group)
 enum { XQ_FULL = 0, XK_FULL = 1, XK_EMPTY = XK_FULL + kXStages, XS_FULL = XK_EMPTY + kXStages,
        XS_EMPTY = XS_FULL + kXBufs, X_NUM_BARS = XS_EMPTY + kXBufs };
+// extract with the sender's own output (O_s = P V_s accumulated in TMEM): a ring of value tiles,
+// two staging buffers per writer group that hold the bf16 P tile the P.V MMA reads, and the
+// completion of the last P.V MMA
+constexpr int kVStages = 3;
+constexpr int kOLag = 2;           // P.V of block t is issued after the QK^T of block t + kOLag
+enum { XV_FULL = X_NUM_BARS, XV_EMPTY = XV_FULL + kVStages, XP_READY = XV_EMPTY + kVStages,
+       XP_FREE = XP_READY + 4, XO_FULL = XP_FREE + 4, XO_NUM_BARS = XO_FULL + 1 };
 
 struct StatsParams {
   CUtensorMap q_map;   // {64, n, H_s * D / 64} bf16, box {64, 128, 1}
@@ -90,6 +97,11 @@ struct ExtractParams {
   int64_t dense_tiles;
   float* norm2;
   float* sum1;
+  // sender output (extract_tc_kernel<D, true>): V_s bf16 viewed {64, n_k, H_s * d_vs / 64}, box
+  // {64, 64, d_vs / 64}; o_s fp32 [n, H_s, d_vs]
+  CUtensorMap vs_map;
+  float* o_s;
+  int d_vs;
 };
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t bars, int i) { return bars + 8u * (uint32_t)i; }
@@ -220,10 +232,12 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
   const int h = blockIdx.x - pair * p.H_s;
   const int2 it = p.tab.pairs[pair];
   const int s = it.x, I0 = it.y, P = I0 >> 1;
-  const int row0 = p.cu[s];                 // packed row index of the sequence's token 0
-  const int seq0 = p.tok0 ? p.tok0[s] : row0;   // its q/k token
-  const int L = p.cu[s + 1] - row0;
+  const int row0 = p.tab.qoff[s];           // packed lse row of the sequence-local row 0
+  const int ktok0 = p.tok0 ? p.tok0[s] : p.cu[s];   // k token of key 0
+  const int qtok0 = p.tok0 ? p.tok0[s] : row0;      // q token of row 0
+  const int L = p.cu[s + 1] - p.cu[s];
   const int nb = p.tab.nb[s];
+  const int Ifirst = p.tab.I0[s];           // first row block of the chunk (0: whole sequence)
   const int nT = P + 1;                     // key tiles of 128
 
   if (tid == 0) {
@@ -251,7 +265,7 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
         tc::mbar_expect_tx(bar_addr(bars, Q_FULL), kQBytes);
 #pragma unroll
         for (int qp = 0; qp < NPAN; ++qp)
-          tc::tma_load_3d(sQ + qp * kPanel128, &p.q_map, 0, seq0 + kRows * P, h * NPAN + qp,
+          tc::tma_load_3d(sQ + qp * kPanel128, &p.q_map, 0, qtok0 + kRows * P, h * NPAN + qp,
                           bar_addr(bars, Q_FULL));
       }
       tc::prefetch_tmap(&p.k_map);
@@ -260,7 +274,7 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
         if (T >= kSStages)
           tc::wait_bar(bar_addr(bars, K_EMPTY + st), ((T / kSStages) - 1) & 1, abort_flag, p.status);
         tc::mbar_expect_tx(bar_addr(bars, K_FULL + st), kPanel128);
-        tc::tma_load_3d(sK + st * kKStage + pan * kPanel128, &p.k_map, 0, seq0 + 128 * T,
+        tc::tma_load_3d(sK + st * kKStage + pan * kPanel128, &p.k_map, 0, ktok0 + 128 * T,
                         h * NPAN + pan, bar_addr(bars, K_FULL + st));
       }
       for (int T = max(0, nT - kSStages); T < nT; ++T)
@@ -295,7 +309,7 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
     const int r = 32 * qd + lane;                 // TMEM lane = pair-local row
     const int Ir = I0 + (r >> 6);                 // row block (uniform over the warp)
     const int i = kRows * P + r;                  // sequence-local row
-    const bool valid = i < L;
+    const bool valid = i < L && Ir >= Ifirst;
     const uint32_t t_lane = (uint32_t)(32 * qd) << 16;
     const float sc = p.scale_log2;
     float m_acc = -INFINITY, l_acc = 0.f;
@@ -384,10 +398,10 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
     for (int idx = tid; idx < 2 * kMaxNb; idx += kSoft) {
       const int k = idx / kMaxNb, J = idx - k * kMaxNb;
       const int I = I0 + k;
-      if (I < nb && J <= I) {
+      if (I < nb && I >= Ifirst && J <= I) {
         const float m = part[(2 * k) * kMaxNb + J] + part[(2 * k + 1) * kMaxNb + J];
         mass_s[k * kMaxNb + J] = m;
-        p.mass[(int64_t)h * p.ncb + p.tab.cb_start[s] + (int64_t)I * (I + 1) / 2 + J] = m;
+        p.mass[(int64_t)h * p.ncb + tab_cb(p.tab, s, I) + J] = m;
       }
     }
     tc::named_bar(1, kSoft);
@@ -398,13 +412,13 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
     if (p.tau >= 1.f) {
       for (int idx = tid; idx < 2 * kMaxNb; idx += kSoft) {
         const int k = idx / kMaxNb, J = idx - k * kMaxNb, I = I0 + k;
-        if (I < nb && J <= I)
-          atomicOr(p.headmask_dense + p.tab.cb_start[s] + (int64_t)I * (I + 1) / 2 + J, bit);
+        if (I < nb && I >= Ifirst && J <= I)
+          atomicOr(p.headmask_dense + tab_cb(p.tab, s, I) + J, bit);
       }
     } else {
       for (int idx = tid; idx < 2 * kMaxNb; idx += kSoft) {
         const int k = idx / kMaxNb, J = idx - k * kMaxNb, I = I0 + k;
-        if (I < nb && J <= I) {
+        if (I < nb && I >= Ifirst && J <= I) {
           const float* ms = mass_s + k * kMaxNb;
           const float mJ = ms[J];
           int rank = 0;
@@ -417,14 +431,15 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
         }
       }
       tc::named_bar(1, kSoft);
-      if (warp < 2 && I0 + warp < nb) warp_exclusive_scan256(sorted_s + warp * kMaxNb, I0 + warp + 1, lane);
+      if (warp < 2 && I0 + warp < nb && I0 + warp >= Ifirst)
+        warp_exclusive_scan256(sorted_s + warp * kMaxNb, I0 + warp + 1, lane);
       tc::named_bar(1, kSoft);
       for (int idx = tid; idx < 2 * kMaxNb; idx += kSoft) {
         const int k = idx / kMaxNb, J = idx - k * kMaxNb, I = I0 + k;
-        if (I < nb && J <= I) {
+        if (I < nb && I >= Ifirst && J <= I) {
           const float R = (float)min(64, L - 64 * I);
           if (sorted_s[k * kMaxNb + rank_s[k * kMaxNb + J]] < p.tau * R)
-            atomicOr(p.headmask_dense + p.tab.cb_start[s] + (int64_t)I * (I + 1) / 2 + J, bit);
+            atomicOr(p.headmask_dense + tab_cb(p.tab, s, I) + J, bit);
         }
       }
     }
@@ -443,21 +458,33 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
 // Stage 2: extraction of the kept tiles
 // ------------------------------------------------------------------------------------------------
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_constant__ ExtractParams p) {
+// OUT: also the sender's own attention output O_s = P V_s (MapFlow news page, the paragraphs on
+// the attention map as the shared state: the sender runs its own attention, the receiver reuses
+// its probabilities). Then every causal column block is visited, not only the kept ones; the
+// bf16 P tile a writer group stages for the stores is also the A operand of a
+// 128 x d_vs x 64 MMA into TMEM columns 256 .. 256 + d_vs, with the value tile as B. The row's
+// final lse is known here, so P is normalised as computed and O_s needs no rescaling.
+template <int D, bool OUT>
+__global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const __grid_constant__ ExtractParams p) {
   constexpr int NPAN = D / 64;
   constexpr uint32_t kQBytes = NPAN * kPanel128;
   constexpr uint32_t kKStage = NPAN * kPanel64;
+  constexpr uint32_t kVStage = 2 * kPanel64;               // room for d_vs up to 128
+  constexpr int kBars = OUT ? XO_NUM_BARS : X_NUM_BARS;
+  constexpr uint32_t kTmemCols = OUT ? 512u : 256u;
+  constexpr int kStageBufs = OUT ? 2 : 1;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase, sK = sbase + kQBytes;
-  unsigned char* stage_all = smem + kQBytes + kXStages * kKStage;        // 8 warps x 4 KB
-  int64_t* base_s = reinterpret_cast<int64_t*>(stage_all + 8 * 4096);    // [2][256] tile index
+  const uint32_t sV = sK + kXStages * kKStage;             // OUT: value-tile ring
+  unsigned char* stage_all = smem + kQBytes + kXStages * kKStage + (OUT ? kVStages * kVStage : 0);
+  // 8 warps x 4 KB per staging buffer
+  int64_t* base_s = reinterpret_cast<int64_t*>(stage_all + kStageBufs * 8 * 4096);   // [2][256]
   int* rk_s = reinterpret_cast<int*>(base_s + 2 * kMaxNb);               // [2][256] rank | k << 8
   int* ulist = rk_s + 2 * kMaxNb;                                        // [256] union of J
   uint64_t* bar_mem = reinterpret_cast<uint64_t*>(ulist + kMaxNb);
-  uint32_t* misc = reinterpret_cast<uint32_t*>(bar_mem + X_NUM_BARS);    // [0] tmem [1] abort [2] count
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bar_mem + kBars);         // [0] tmem [1] abort [2] count
   const uint32_t bars = smem_u32(bar_mem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
@@ -466,20 +493,26 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
   const int h = blockIdx.x - pair * p.H_s;
   const int2 it = p.tab.pairs[pair];
   const int s = it.x, I0 = it.y, P = I0 >> 1;
-  const int row0 = p.cu[s];
-  const int seq0 = p.tok0 ? p.tok0[s] : row0;
-  const int L = p.cu[s + 1] - row0;
+  const int row0 = p.tab.qoff[s];           // packed lse row of the sequence-local row 0
+  const int ktok0 = p.tok0 ? p.tok0[s] : p.cu[s];
+  const int qtok0 = p.tok0 ? p.tok0[s] : row0;
+  const int L = p.cu[s + 1] - p.cu[s];
   const int nb = p.tab.nb[s];
+  const int Ifirst = p.tab.I0[s];
   const int nJ = min(2 * P + 2, nb);
 
   if (tid == 0) {
-    for (int i = 0; i < X_NUM_BARS; ++i)
-      tc::mbar_init(bar_addr(bars, i), (i >= XS_EMPTY && i < XS_EMPTY + kXBufs) ? 4u : 1u);
+    for (int i = 0; i < kBars; ++i) {
+      uint32_t cnt = 1;
+      if (i >= XS_EMPTY && i < XS_EMPTY + kXBufs) cnt = 4;
+      if (OUT && i >= XP_READY && i < XP_READY + 4) cnt = 4;
+      tc::mbar_init(bar_addr(bars, i), cnt);
+    }
     misc[1] = 0;
     tc::fence_barrier_init();
   }
   for (int idx = tid; idx < 2 * kMaxNb; idx += kThreads) base_s[idx] = -1;
-  if (warp == 9) tc::tmem_alloc(smem_u32(misc), 256);
+  if (warp == 9) tc::tmem_alloc(smem_u32(misc), kTmemCols);
   __syncthreads();
   // this head's stored blocks in row blocks I0 and I1, by column block
   if (p.dense) {
@@ -490,8 +523,8 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
         rk_s[idx] = 1 << 8;
       }
     }
-  } else if (warp < 2 && I0 + warp < nb) {
-    const int rb = p.tab.rb_start[s] + I0 + warp;
+  } else if (warp < 2 && I0 + warp < nb && I0 + warp >= Ifirst) {
+    const int rb = tab_rb(p.tab, s, I0 + warp);
     const int u0 = p.row_ptr[rb], u1 = p.row_ptr[rb + 1];
     const unsigned long long below = (1ull << h) - 1ull;
     for (int u = u0 + lane; u < u1; u += 32) {
@@ -505,10 +538,11 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
   }
   __syncthreads();
   if (warp == 0) {
+    // the column blocks to visit: the union of the kept ones, or (OUT) all causal ones
     int cnt = 0;
     for (int J0 = 0; J0 < nJ; J0 += 32) {
       const int J = J0 + lane;
-      const bool any = J < nJ && (base_s[J] >= 0 || base_s[kMaxNb + J] >= 0);
+      const bool any = J < nJ && (OUT || base_s[J] >= 0 || base_s[kMaxNb + J] >= 0);
       const unsigned bal = __ballot_sync(0xffffffffu, any);
       if (any) ulist[cnt + __popc(bal & ((1u << lane) - 1u))] = J;
       cnt += __popc(bal);
@@ -525,10 +559,12 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
     if (lane == 0) {
       tc::prefetch_tmap(&p.q_map);
       tc::prefetch_tmap(&p.k_map);
+      if (OUT) tc::prefetch_tmap(&p.vs_map);
+      const uint32_t vbytes = OUT ? (uint32_t)p.d_vs * 128u : 0u;
       tc::mbar_expect_tx(bar_addr(bars, XQ_FULL), kQBytes);
 #pragma unroll
       for (int pan = 0; pan < NPAN; ++pan)
-        tc::tma_load_3d(sQ + pan * kPanel128, &p.q_map, 0, seq0 + kRows * P, h * NPAN + pan,
+        tc::tma_load_3d(sQ + pan * kPanel128, &p.q_map, 0, qtok0 + kRows * P, h * NPAN + pan,
                         bar_addr(bars, XQ_FULL));
       for (int t = 0; t < nU; ++t) {
         const int st = t % kXStages;
@@ -538,16 +574,48 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
         const int J = ulist[t];
 #pragma unroll
         for (int pan = 0; pan < NPAN; ++pan)
-          tc::tma_load_3d(sK + st * kKStage + pan * kPanel64, &p.k_map, 0, seq0 + 64 * J,
+          tc::tma_load_3d(sK + st * kKStage + pan * kPanel64, &p.k_map, 0, ktok0 + 64 * J,
                           h * NPAN + pan, bar_addr(bars, XK_FULL + st));
+        if (OUT) {
+          // value tile of block t (both 64-dim halves in one box); its slot is free once the
+          // P.V MMA of block t - kVStages completed
+          const int vs = t % kVStages;
+          if (t >= kVStages)
+            tc::wait_bar(bar_addr(bars, XV_EMPTY + vs), ((t / kVStages) - 1) & 1, abort_flag, p.status);
+          tc::mbar_expect_tx(bar_addr(bars, XV_FULL + vs), vbytes);
+          tc::tma_load_3d(sV + vs * kVStage, &p.vs_map, 0, ktok0 + 64 * J, h * (p.d_vs / 64),
+                          bar_addr(bars, XV_FULL + vs));
+        }
       }
       for (int t = max(0, nU - kXStages); t < nU; ++t)
         tc::drain_bar(bar_addr(bars, XK_FULL + t % kXStages), (t / kXStages) & 1);
+      if (OUT)
+        for (int t = max(0, nU - kVStages); t < nU; ++t)
+          tc::drain_bar(bar_addr(bars, XV_FULL + t % kVStages), (t / kVStages) & 1);
       tc::drain_bar(bar_addr(bars, XQ_FULL), 0);
     }
   } else if (warp == 9) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(128, 64, 0, 0);
+      // O_s += P_t . V_s[J_t]: P from the staging buffer of block t's writer group (K-major,
+      // 128 rows x 64 keys), V MN-major (d_vs columns per key; the second 64-dim half 8 KB on)
+      auto issue_pv = [&](int t) {
+        const int G = t & 1, c = t >> 1, sb = c & 1, u = c >> 1, vs = t % kVStages;
+        tc::wait_bar(bar_addr(bars, XP_READY + 2 * G + sb), u & 1, abort_flag, p.status);
+        tc::wait_bar(bar_addr(bars, XV_FULL + vs), (t / kVStages) & 1, abort_flag, p.status);
+        tc::tc_fence_after();
+        const uint32_t pa = smem_u32(stage_all) + (uint32_t)(sb * 8 + 4 * G) * 4096u;
+        const uint32_t va = sV + (uint32_t)vs * kVStage;
+        const uint32_t id_pv = tc::idesc_bf16(128, p.d_vs, 0, 1);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t a = tc::sdesc_sw128(pa + kk * 32u, 16u, 1024u);
+          const uint64_t b = tc::sdesc_sw128(va + kk * 2048u, 8192u, 1024u);
+          tc::mma_bf16(tmem + 256u, a, b, id_pv, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(bar_addr(bars, XP_FREE + 2 * G + sb));
+        tc::mma_commit(bar_addr(bars, XV_EMPTY + vs));
+      };
       tc::wait_bar(bar_addr(bars, XQ_FULL), 0, abort_flag, p.status);
       for (int t = 0; t < nU; ++t) {
         const int st = t % kXStages, b = t & (kXBufs - 1);
@@ -563,8 +631,15 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
         }
         tc::mma_commit(bar_addr(bars, XK_EMPTY + st));
         tc::mma_commit(bar_addr(bars, XS_FULL + b));
+        if (OUT && t >= kOLag) issue_pv(t - kOLag);
       }
-      if (nU > 0) tc::drain_bar(bar_addr(bars, XS_FULL + ((nU - 1) & (kXBufs - 1))), ((nU - 1) >> 2) & 1);
+      if (OUT) {
+        for (int t = max(0, nU - kOLag); t < nU; ++t) issue_pv(t);
+        tc::mma_commit(bar_addr(bars, XO_FULL));
+        tc::drain_bar(bar_addr(bars, XO_FULL), 0);
+      } else if (nU > 0) {
+        tc::drain_bar(bar_addr(bars, XS_FULL + ((nU - 1) & (kXBufs - 1))), ((nU - 1) >> 2) & 1);
+      }
     }
   } else {
     // ------------------------------ writers: group G takes the blocks t = G, G + 2, ... --------
@@ -573,23 +648,26 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
     const int kb = r >> 6;                        // 0: row block I0, 1: I1 (uniform over the warp)
     const int Ir = I0 + kb;
     const int i = kRows * P + r;
-    const bool valid = i < L;
+    const bool valid = i < L && Ir >= Ifirst;
     const int il = r & 63;                        // row within the tile
     const uint32_t t_lane = (uint32_t)(32 * qd) << 16;
     const float sc = p.scale_log2;
     const float lse2 = valid ? p.lse[(int64_t)h * p.n + row0 + i] * kLog2e : 0.f;
-    unsigned char* stg = stage_all + warp * 4096;
     bool cap_flag = false;
     float acc1 = 0.f, acc2 = 0.f;   // dense mode: sum and squared norm of this row's rounded values
     for (int t = G; t < nU; t += 2) {
       const int b = t & (kXBufs - 1);
+      const int c = t >> 1, sb = OUT ? (c & 1) : 0;
+      unsigned char* stg = stage_all + (sb * 8 + warp) * 4096;
       tc::wait_bar(bar_addr(bars, XS_FULL + b), (t >> 2) & 1, abort_flag, p.status);
       tc::tc_fence_after();
       const int J = ulist[t];
       const int64_t base = base_s[kb * kMaxNb + J];
       const int rk = rk_s[kb * kMaxNb + J];
       const int rank = rk & 255, k = rk >> 8;
-      if (base >= 0) {
+      // OUT: every block feeds the P.V MMA, so every block's P is staged
+      const bool stage = OUT || base >= 0;
+      if (stage) {
         // exp(s - lse) of this row, 32 columns at a time, staged as bf16 (16-byte chunk c of
         // the row at c ^ (row & 7))
         const int j0 = 64 * J;
@@ -598,6 +676,8 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
         IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(b * 64), v);
         IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(b * 64 + 32), (v + 32));
         tc::tmem_ld_wait();
+        if (OUT && c >= 2)   // the P.V MMA of this buffer's previous block has read it
+          tc::wait_bar(bar_addr(bars, XP_FREE + 2 * G + sb), ((c >> 1) - 1) & 1, abort_flag, p.status);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[16];
@@ -632,28 +712,34 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
             }
           }
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int cc = 4 * half + c;
+          for (int cq = 0; cq < 4; ++cq) {
+            const int cc = 4 * half + cq;
             *reinterpret_cast<uint4*>(stg + lane * 128 + ((cc ^ (lane & 7)) << 4)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                make_uint4(pk[4 * cq], pk[4 * cq + 1], pk[4 * cq + 2], pk[4 * cq + 3]);
           }
         }
       }
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar_addr(bars, XS_EMPTY + b));
+      if (OUT) {
+        // the staged tile goes to the tensor cores (async proxy) as well as to the stores below
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar_addr(bars, XP_READY + 2 * G + sb));
+      }
       if (base < 0) continue;
       // write 4 tile rows of 128 B per step
       __syncwarp();
       if (base + k <= p.capacity) {
         __nv_bfloat16* blk = p.vals + base * (64 * 64) + (int64_t)rank * 64;
-        const int c = lane & 7;
+        const int cl = lane & 7;
 #pragma unroll
         for (int step = 0; step < 8; ++step) {
           const int row = 4 * step + (lane >> 3);          // warp-local row
-          const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 128 + ((c ^ (row & 7)) << 4));
+          const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 128 + ((cl ^ (row & 7)) << 4));
           const int tr = (il - lane) + row;                 // tile row of that warp-local row
-          *reinterpret_cast<uint4*>(blk + (int64_t)tr * k * 64 + c * 8) = val;
+          *reinterpret_cast<uint4*>(blk + (int64_t)tr * k * 64 + cl * 8) = val;
         }
       } else {
         cap_flag = true;
@@ -672,13 +758,44 @@ __global__ void __launch_bounds__(kThreads, 2) extract_tc_kernel(const __grid_co
         atomicAdd(p.norm2 + (int64_t)s * p.H_s + h, acc2);
       }
     }
+    if (OUT) {
+      // O_s rows out of TMEM: group G takes columns [G * d_vs / 2, (G + 1) * d_vs / 2), 32 at a
+      // time, transposed through this warp's staging slice so that each row leaves as 128-byte
+      // runs (4 rows per store instruction)
+      tc::wait_bar(bar_addr(bars, XO_FULL), 0, abort_flag, p.status);
+      tc::tc_fence_after();
+      const int half_cols = p.d_vs / 2;
+      float* scr = reinterpret_cast<float*>(stage_all + warp * 4096);   // [32 rows][32 floats]
+      for (int c0 = G * half_cols; c0 < (G + 1) * half_cols; c0 += 32) {
+        uint32_t v[32];
+        IAMAP_TMEM_LD32(tmem + t_lane + 256u + (uint32_t)c0, v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int cq = 0; cq < 8; ++cq)
+          *reinterpret_cast<uint4*>(scr + lane * 32 + ((cq ^ (lane & 7)) << 2)) =
+              make_uint4(v[4 * cq], v[4 * cq + 1], v[4 * cq + 2], v[4 * cq + 3]);
+        __syncwarp();
+        const int cl = lane & 7;
+#pragma unroll
+        for (int step = 0; step < 8; ++step) {
+          const int row = 4 * step + (lane >> 3);           // warp-local row
+          const int ir = kRows * P + 32 * qd + row;         // its sequence-local row
+          const int Irr = I0 + ((32 * qd + row) >> 6);
+          if (ir < L && Irr >= Ifirst) {
+            const uint4 val = *reinterpret_cast<const uint4*>(scr + row * 32 + ((cl ^ (row & 7)) << 2));
+            *reinterpret_cast<uint4*>(p.o_s + ((int64_t)(row0 + ir) * p.H_s + h) * p.d_vs + c0 + 4 * cl) = val;
+          }
+        }
+        __syncwarp();
+      }
+    }
   }
 
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 9) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, 256);
+    tc::tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -688,10 +805,12 @@ static size_t stats_smem() {
          sizeof(float) * (2 * kRows + 2 * kRows + kRows + 4 * kMaxNb + 2 * kMaxNb + 2 * kMaxNb) +
          sizeof(int) * 2 * kMaxNb + 8 * NUM_BARS + 16;
 }
-template <int D>
+template <int D, bool OUT>
 static size_t extract_smem() {
-  return 1024 + (size_t)(D / 64) * (kPanel128 + kXStages * kPanel64) + 8 * 4096 +
-         sizeof(int64_t) * 2 * kMaxNb + sizeof(int) * 3 * kMaxNb + 8 * X_NUM_BARS + 16;
+  return 1024 + (size_t)(D / 64) * (kPanel128 + kXStages * kPanel64) +
+         (OUT ? (size_t)kVStages * 2 * kPanel64 + 2 * 8 * 4096 : 8 * 4096) +
+         sizeof(int64_t) * 2 * kMaxNb + sizeof(int) * 3 * kMaxNb +
+         8 * (OUT ? XO_NUM_BARS : X_NUM_BARS) + 16;
 }
 
 }  // namespace tccomp
@@ -709,8 +828,9 @@ int compress_stats_tc_launch(const CompressArgs& a, cudaStream_t stream) {
   using namespace tccomp;
   StatsParams p{};
   const int64_t n_tok = a.n_tok > 0 ? a.n_tok : a.n;
+  const int64_t n_key = a.n_k > 0 ? a.n_k : n_tok;
   int rc = encode_qk_map(&p.q_map, a.q, n_tok, a.H_s, a.d, 128);
-  if (!rc) rc = encode_qk_map(&p.k_map, a.k, n_tok, a.H_s, a.d, 128);
+  if (!rc) rc = encode_qk_map(&p.k_map, a.k, n_key, a.H_s, a.d, 128);
   if (rc) return rc;
   p.cu = a.cu_seqlens;
   p.tok0 = a.tok0;
@@ -742,8 +862,9 @@ int compress_extract_tc_launch(const CompressArgs& a, cudaStream_t stream) {
   using namespace tccomp;
   ExtractParams p{};
   const int64_t n_tok = a.n_tok > 0 ? a.n_tok : a.n;
+  const int64_t n_key = a.n_k > 0 ? a.n_k : n_tok;
   int rc = encode_qk_map(&p.q_map, a.q, n_tok, a.H_s, a.d, 128);
-  if (!rc) rc = encode_qk_map(&p.k_map, a.k, n_tok, a.H_s, a.d, 64);
+  if (!rc) rc = encode_qk_map(&p.k_map, a.k, n_key, a.H_s, a.d, 64);
   if (rc) return rc;
   p.cu = a.cu_seqlens;
   p.tok0 = a.tok0;
@@ -765,8 +886,20 @@ int compress_extract_tc_launch(const CompressArgs& a, cudaStream_t stream) {
   p.vals = static_cast<__nv_bfloat16*>(a.vals);
   p.capacity = a.capacity;
   p.status = a.status;
-  const size_t smem = a.d == 64 ? extract_smem<64>() : extract_smem<128>();
-  auto kern = a.d == 64 ? extract_tc_kernel<64> : extract_tc_kernel<128>;
+  const bool out = a.o_s != nullptr;
+  if (out) {
+    if (a.dense || !a.v_s || (a.d_vs != 64 && a.d_vs != 128))
+      return set_error(IAMAP_ERR_INVALID_ARG, "sender output needs v_s and d_vs of 64 or 128");
+    rc = encode_tmap_3d_bf16(&p.vs_map, a.v_s, 64, (uint64_t)n_key, (uint64_t)a.H_s * (a.d_vs / 64),
+                             (uint64_t)a.H_s * a.d_vs * 2, 128, 64, 64, (uint32_t)(a.d_vs / 64));
+    if (rc) return rc;
+    p.o_s = a.o_s;
+    p.d_vs = a.d_vs;
+  }
+  const size_t smem = out ? (a.d == 64 ? extract_smem<64, true>() : extract_smem<128, true>())
+                          : (a.d == 64 ? extract_smem<64, false>() : extract_smem<128, false>());
+  auto kern = out ? (a.d == 64 ? extract_tc_kernel<64, true> : extract_tc_kernel<128, true>)
+                  : (a.d == 64 ? extract_tc_kernel<64, false> : extract_tc_kernel<128, false>);
   IAMAP_CUDA_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const int64_t grid = a.plan.num_pairs * a.H_s;
   if (grid > 0) {

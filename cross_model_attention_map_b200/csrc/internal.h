@@ -42,6 +42,14 @@ struct CompressArgs {
   // with per-head sums and squared norms.
   const int32_t* tok0 = nullptr;
   int64_t n_tok = 0;
+  // Chunked prefill: k holds n_k key tokens packed by cu_seqlens (the keys [0, e) of every
+  // sequence), q the n query rows of the chunks (SeqTables::qoff); 0 = q and k alike.
+  int64_t n_k = 0;
+  // Sender output (extract only): v_s bf16 [n_k, H_s, d_vs] packed like k; o_s fp32
+  // [n, H_s, d_vs] packed like q. Null: no sender output.
+  const void* v_s = nullptr;
+  int d_vs = 0;
+  float* o_s = nullptr;
   int dense = 0;
   int64_t dense_tiles = 0;
   float* norm2 = nullptr;
@@ -78,6 +86,9 @@ struct MappedAvArgs {
   int d_v = 0;
   float* out = nullptr;
   unsigned int* status = nullptr;
+  // Chunked prefill: v holds n_k tokens packed by cu_seqlens (the keys of every sequence), out
+  // the n query rows of the chunks (SeqTables::qoff); 0 = v and out alike.
+  int64_t n_k = 0;
 };
 int mapped_av_impl(const MappedAvArgs& a, cudaStream_t stream);
 // Tensor-core, cluster-cooperative form (mapped_av_tc.cu); used when supported.

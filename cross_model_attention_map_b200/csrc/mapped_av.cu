@@ -66,9 +66,10 @@ __global__ void __launch_bounds__(kAvThreads, 1) mapped_av_kernel(AvParams p) {
   const int grp = blockIdx.x - item * p.groups;
   const int2 it = p.tab.items[item];
   const int s = it.x, I = it.y;
-  const int seq0 = p.cu[s];
+  const int seq0 = p.cu[s];                 // V token of key 0
+  const int orow0 = p.tab.qoff[s];          // output row of the sequence-local row 0
   const int L = p.cu[s + 1] - seq0;
-  const int rb = p.tab.rb_start[s] + I;
+  const int rb = tab_rb(p.tab, s, I);
   const int r0 = grp * kAvGroup;
   const int G = min(kAvGroup, p.H_r - r0);
   const int64_t vrs = (int64_t)p.H_kv * DV;  // V row stride (elements)
@@ -215,7 +216,7 @@ __global__ void __launch_bounds__(kAvThreads, 1) mapped_av_kernel(AvParams p) {
     for (int hr = 0; hr < 2; ++hr) {
       const int i = I * kT + pv_rows + g + 8 * hr;
       if (i < L) {
-        float* dst = p.out + ((int64_t)(seq0 + i) * p.H_r + r) * DV;
+        float* dst = p.out + ((int64_t)(orow0 + i) * p.H_r + r) * DV;
 #pragma unroll
         for (int nt = 0; nt < DV / 8; ++nt)
           *reinterpret_cast<float2*>(dst + nt * 8 + 2 * t4) =

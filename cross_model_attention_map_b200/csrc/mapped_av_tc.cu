@@ -105,6 +105,10 @@ constexpr int kMaxNP = 12;       // sender-slice ring: as many slots as shared m
 // spread over several producer warps: four for the sender slices (chunks round-robin) and one
 // per receiver head for the V tiles (each a single 3-D box of both 64-dim halves).
 constexpr int kPWarps = 4, kVWarps = 4;
+// The sender slices of the block kPrefetch ahead are prefetched into L2 (by the warp that will
+// load each chunk), so that the ring's loads find them there: the ring holds only ~1.5 blocks,
+// too few bytes in flight to cover the HBM latency on its own.
+constexpr int kPrefetch = 3;
 constexpr int kND = 8;           // mixing-result TMEM slots (chunks)
 constexpr int kNG = kND / 2;     // ... committed and released in pairs of chunks (one commit costs
                                  // ~90 ns of issue time on this B200, an MMA ~25 ns)
@@ -160,9 +164,10 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
   const int item = blockIdx.x / C;
   const int2 it = p.tab.items[item];
   const int s = it.x, I = it.y;
-  const int seq0 = p.cu[s];
+  const int seq0 = p.cu[s];                 // V token of key 0
+  const int orow0 = p.tab.qoff[s];          // output row of the sequence-local row 0
   const int L = p.cu[s + 1] - seq0;
-  const int rb = p.tab.rb_start[s] + I;
+  const int rb = tab_rb(p.tab, s, I);
   const int u0 = p.row_ptr[rb];
   const int T = p.row_ptr[rb + 1] - u0;
   const int r0 = (int)crank * kG;
@@ -212,9 +217,23 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
       const uint64_t pol = tc::policy_evict_first();   // each stored tile is read once
       if (pw == 0)
         for (int i = 0; i < 8; ++i) tc::prefetch_tmap(&p.p_maps[i]);
+      // L2 prefetch of this warp's chunks of block tb
+      auto prefetch_block = [&](int tb) {
+        const unsigned long long mp = p.headmask[u0 + tb];
+        const int kp = __popcll(mp);
+        const int yp = (int)(p.val_off[u0 + tb] * 64);
+        const CUtensorMap* mapp = &p.p_maps[((kp + 7) >> 3) - 1];
+        for (int c = 0; c < nch; ++c) {
+          if ((tb * nch + c) % kPWarps != pw) continue;
+          tc::tma_prefetch_2d(mapp, 0, yp + (2 * (c0 + c)) * kp);
+          tc::tma_prefetch_2d(mapp, 0, yp + (2 * (c0 + c) + 1) * kp);
+        }
+      };
+      for (int tb = 1; tb <= kPrefetch && tb < T; ++tb) prefetch_block(tb);
       unsigned long long m_next = T > 0 ? p.headmask[u0] : 0ull;
       int64_t off_next = T > 0 ? p.val_off[u0] : 0;
       for (int t = 0; t < T; ++t) {
+        if (t + kPrefetch + 1 < T) prefetch_block(t + kPrefetch + 1);
         const unsigned long long m = m_next;
         const int64_t off = off_next;
         if (t + 1 < T) {
@@ -466,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
           uint32_t v[32];
           IAMAP_TMEM_LD32(tmem + lane_base + (uint32_t)(rl * 64 + half * 32), v);
           tc::tmem_ld_wait();
-          float* o = p.out + ((int64_t)(seq0 + I * 64 + half * 32) * p.H_r + r0 + rl) * p.d_v + dv;
+          float* o = p.out + ((int64_t)(orow0 + I * 64 + half * 32) * p.H_r + r0 + rl) * p.d_v + dv;
 #pragma unroll
           for (int ii = 0; ii < 32; ++ii)
             if (I * 64 + half * 32 + ii < L)
@@ -549,7 +568,8 @@ int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream) {
   }
   const int H_kv = a.H_kv > 0 ? a.H_kv : a.H_r;
   p.grp = a.H_r / H_kv;
-  int rc = encode_tmap_3d_bf16(&p.v_map, a.v, 64, (uint64_t)a.n, (uint64_t)H_kv * (a.d_v / 64),
+  const int64_t n_v = a.n_k > 0 ? a.n_k : a.n;
+  int rc = encode_tmap_3d_bf16(&p.v_map, a.v, 64, (uint64_t)n_v, (uint64_t)H_kv * (a.d_v / 64),
                                (uint64_t)H_kv * a.d_v * 2, 128, 64, 64, (uint32_t)(a.d_v / 64));
   if (rc) return rc;
   p.cu = a.cu_seqlens;

@@ -87,10 +87,50 @@ int make_plan(const int32_t* cu_host, int num_seqs, int B, int64_t n, Plan* out)
   return IAMAP_OK;
 }
 
+int make_chunk_plan(const int32_t* cu_k_host, const int32_t* cu_q_host,
+                    const int32_t* starts_host, int num_seqs, int B, int64_t n_k, int64_t n_q,
+                    Plan* out) {
+  if (!cu_k_host || !cu_q_host || !starts_host)
+    return set_error(IAMAP_ERR_INVALID_ARG, "cu_k_host, cu_q_host and starts_host are required");
+  if (num_seqs < 1) return set_error(IAMAP_ERR_INVALID_ARG, "num_seqs must be >= 1");
+  if (B < 1) return set_error(IAMAP_ERR_INVALID_ARG, "block size must be >= 1");
+  if (cu_k_host[0] != 0 || cu_q_host[0] != 0)
+    return set_error(IAMAP_ERR_INVALID_ARG, "cu_k[0] and cu_q[0] must be 0");
+  Plan p;
+  for (int s = 0; s < num_seqs; ++s) {
+    const int64_t e = (int64_t)cu_k_host[s + 1] - cu_k_host[s];
+    const int64_t rows = (int64_t)cu_q_host[s + 1] - cu_q_host[s];
+    const int64_t c0 = starts_host[s];
+    if (e < 0 || rows < 0) return set_error(IAMAP_ERR_INVALID_ARG, "cu_k or cu_q decreases at %d", s);
+    if (c0 < 0 || c0 % B != 0)
+      return set_error(IAMAP_ERR_INVALID_ARG, "chunk start %lld of sequence %d is not a "
+                       "non-negative multiple of B=%d", (long long)c0, s, B);
+    if (c0 + rows != e)
+      return set_error(IAMAP_ERR_INVALID_ARG, "sequence %d: a chunk of %lld query rows from %lld "
+                       "does not end at the key length %lld", s, (long long)rows, (long long)c0,
+                       (long long)e);
+    const int64_t nb = (e + B - 1) / B, i0 = c0 / B;
+    if (i0 < nb) {
+      p.num_rowblocks += nb - i0;
+      p.num_causal_blocks += nb * (nb + 1) / 2 - i0 * (i0 + 1) / 2;
+      p.num_pairs += (nb + 1) / 2 - i0 / 2;
+    }
+    if (nb > p.max_nb) p.max_nb = (int32_t)nb;
+  }
+  if ((int64_t)cu_k_host[num_seqs] != n_k || (int64_t)cu_q_host[num_seqs] != n_q)
+    return set_error(IAMAP_ERR_INVALID_ARG, "cu_k / cu_q totals (%d, %d) differ from n_k=%lld, "
+                     "n_q=%lld", cu_k_host[num_seqs], cu_q_host[num_seqs], (long long)n_k,
+                     (long long)n_q);
+  if (p.num_causal_blocks >= (int64_t)INT32_MAX)
+    return set_error(IAMAP_ERR_UNSUPPORTED, "more than 2^31 causal blocks");
+  *out = p;
+  return IAMAP_OK;
+}
+
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t seq_tables_bytes(int num_seqs, int64_t num_rowblocks) {
-  return align256(sizeof(int32_t) * (size_t)num_seqs) +
+  return 3 * align256(sizeof(int32_t) * (size_t)num_seqs) +
          2 * align256(sizeof(int32_t) * (size_t)(num_seqs + 1)) +
          align256(sizeof(int2) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1)) +
          align256(sizeof(int64_t) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1)) +
@@ -111,55 +151,71 @@ SeqTables carve_seq_tables(void* ws, int num_seqs, int64_t num_rowblocks) {
   t.row_tiles = reinterpret_cast<int64_t*>(p);
   p += align256(sizeof(int64_t) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1));
   t.pairs = reinterpret_cast<int2*>(p);   // at most num_rowblocks pairs
+  p += align256(sizeof(int2) * (size_t)(num_rowblocks > 0 ? num_rowblocks : 1));
+  t.I0 = reinterpret_cast<int32_t*>(p);
+  p += align256(sizeof(int32_t) * (size_t)num_seqs);
+  t.qoff = reinterpret_cast<int32_t*>(p);
   return t;
 }
 
 // One CTA. Row blocks are ordered by decreasing causal length (I descending), then by sequence,
-// so that the longest rows start first (load balance of the triangular work).
+// so that the longest rows start first (load balance of the triangular work). A sequence lists
+// its row blocks I0[s] .. nb[s] - 1 (I0 = 0 without chunks), and the pairs (E, E + 1), E even,
+// that hold at least one of them.
 __global__ void build_tables_kernel(const int32_t* __restrict__ cu, int num_seqs, int B,
-                                    int32_t max_nb, SeqTables t) {
+                                    int32_t max_nb, SeqTables t, const int32_t* __restrict__ cu_q,
+                                    const int32_t* __restrict__ starts) {
   if (threadIdx.x == 0) {
     int32_t rb = 0, cb = 0;
     for (int s = 0; s < num_seqs; ++s) {
       int32_t L = cu[s + 1] - cu[s];
       int32_t nb = (L + B - 1) / B;
+      int32_t i0 = starts ? starts[s] / B : 0;
+      if (i0 > nb) i0 = nb;
       t.nb[s] = nb;
+      t.I0[s] = i0;
+      t.qoff[s] = starts ? cu_q[s] - starts[s] : cu[s];
       t.rb_start[s] = rb;
       t.cb_start[s] = cb;
-      rb += nb;
-      cb += nb * (nb + 1) / 2;
+      rb += nb - i0;
+      cb += nb * (nb + 1) / 2 - i0 * (i0 + 1) / 2;
     }
     t.rb_start[num_seqs] = rb;
     t.cb_start[num_seqs] = cb;
   }
   __syncthreads();
   for (int I = threadIdx.x; I < max_nb; I += blockDim.x) {
+    // items with a longer row block come first
     int32_t base = 0;
     for (int s = 0; s < num_seqs; ++s) {
-      int32_t e = t.nb[s] - 1 - I;
-      base += e > 0 ? e : 0;
+      const int32_t lo = max(t.I0[s], I + 1);
+      base += max(0, t.nb[s] - lo);
     }
     int32_t c = 0;
     for (int s = 0; s < num_seqs; ++s)
-      if (t.nb[s] > I) t.items[base + c++] = make_int2(s, I);
+      if (t.nb[s] > I && I >= t.I0[s]) t.items[base + c++] = make_int2(s, I);
     // pairs (I, I + 1) with I even, in the same order: the pairs after it are those with a
     // larger even first row block
     if ((I & 1) == 0) {
       int32_t pbase = 0;
       for (int s = 0; s < num_seqs; ++s) {
-        const int32_t e = t.nb[s] - 1 - I;
-        pbase += e > 0 ? e / 2 : 0;
+        const int32_t lo = max(I + 2, t.I0[s] & ~1);     // first even block of a later pair
+        const int32_t hi = (t.nb[s] - 1) & ~1;           // last even block of the sequence
+        pbase += hi >= lo ? (hi - lo) / 2 + 1 : 0;
       }
       int32_t pc = 0;
       for (int s = 0; s < num_seqs; ++s)
-        if (t.nb[s] > I) t.pairs[pbase + pc++] = make_int2(s, I);
+        if (t.nb[s] > I && I >= (t.I0[s] & ~1)) t.pairs[pbase + pc++] = make_int2(s, I);
     }
   }
 }
 
 int launch_build_tables(const int32_t* cu_seqlens, int num_seqs, int B, int32_t max_nb,
-                        SeqTables t, cudaStream_t stream) {
-  build_tables_kernel<<<1, 256, 0, stream>>>(cu_seqlens, num_seqs, B, max_nb, t);
+                        SeqTables t, cudaStream_t stream, const int32_t* cu_q,
+                        const int32_t* starts) {
+  if ((cu_q == nullptr) != (starts == nullptr))
+    return set_error(IAMAP_ERR_INVALID_ARG, "chunk tables need both cu_q and starts");
+  build_tables_kernel<<<1, 256, 0, stream>>>(cu_seqlens, num_seqs, B, max_nb, t, cu_q, starts);
   IAMAP_LAUNCH_CHECK("build_tables_kernel");
   return IAMAP_OK;
 }

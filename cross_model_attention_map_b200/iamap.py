@@ -78,6 +78,20 @@ _SIGS = {
     "iamap_prefix_index_clear": (_I, [_P, _P, _I64, _P]),
     "iamap_prefix_insert": (_I, [_P, _P, _I64, _P, _P, _I64, _P, _P]),
     "iamap_prefix_lookup": (_I, [_P, _I64, _P, _I, _P, _P, _I64, _P, _P, _P]),
+    "iamap_prefill_io_bytes": (_SZ, [_I64, _I, _I, _I, _I, _I]),
+    "iamap_prefill_steps_host": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I,
+                                      _I, _I, _F, _I, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                      _I64, _P, _SZ, _P, _SZ, _P]),
+    "iamap_compress_with_output": (_I, [_P, _P, _P, _P, _I, _I64, _I, _I, _I, _F, _I, _F,
+                                        _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64,
+                                        _P, _SZ, _P]),
+    "iamap_chunk_plan": (_I, [_P, _P, _P, _I, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
+                              ctypes.POINTER(ctypes.c_int32)]),
+    "iamap_compress_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I64, _I64, _I, _I, _I,
+                                  _F, _I, _F, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                  _I64, _P, _SZ, _P]),
+    "iamap_mapped_av_chunk": (_I, [_P, _P, _P, _P, _P, _P, _I, _I64, _I64, _I, _I, _P, _P, _P,
+                                   _P, _P, _I64, _P, _I, _I, _P, _I, _P, _P, _SZ, _P]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -193,6 +207,92 @@ def iamap_mapped_av(cu_seqlens, cu_seqlens_host, num_seqs, n, B, H_s, row_ptr, c
         _ptr(val_off), _ptr(vals), vals_capacity_tiles, _ptr(W), H_r, _ptr(v), d_v, _ptr(out),
         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
     del keep
+
+
+def iamap_compress_with_output(q, k, cu_seqlens, cu_seqlens_host, num_seqs, n, H_s, d, B, tau,
+                               bias_window, bias_value, v_s, d_vs, o_s, lse, mass,
+                               headmask_dense, row_ptr, col_idx, headmask, val_off, counts, vals,
+                               vals_capacity_tiles, ws, stream=None):
+    cp, keep = _host_i32(cu_seqlens_host)
+    _check("iamap_compress_with_output", _lib.iamap_compress_with_output(
+        _ptr(q), _ptr(k), _ptr(cu_seqlens), cp, num_seqs, n, H_s, d, B, tau, bias_window,
+        bias_value, _ptr(v_s), d_vs, _ptr(o_s), _ptr(lse), _ptr(mass), _ptr(headmask_dense),
+        _ptr(row_ptr), _ptr(col_idx), _ptr(headmask), _ptr(val_off), _ptr(counts), _ptr(vals),
+        vals_capacity_tiles, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def iamap_prefill_io_bytes(n, H_s, d, H_r, H_kv, d_v) -> int:
+    return _lib.iamap_prefill_io_bytes(n, H_s, d, H_r, H_kv, d_v)
+
+
+def _host_ptrs(tensors):
+    """ctypes array of the data pointers of host tensors (pinned CPU tensors)."""
+    for t in tensors:
+        if t.is_cuda:
+            raise ValueError("host buffers expected")
+    return (ctypes.c_void_p * len(tensors))(*[t.data_ptr() for t in tensors])
+
+
+def iamap_prefill_steps_host(q_host, k_host, v_host, W_host, out_host, cu_seqlens,
+                             cu_seqlens_host, num_seqs, n, H_s, d, H_r, H_kv, d_v, B, tau,
+                             bias_window, bias_value, lse, mass, headmask_dense, row_ptr, col_idx,
+                             headmask, val_off, counts, vals, vals_capacity_tiles, io, ws,
+                             stream=None):
+    """q_host .. out_host: lists (one entry per step) of CPU tensors (pinned for overlap)."""
+    steps = len(q_host)
+    if not (len(k_host) == len(v_host) == len(W_host) == len(out_host) == steps):
+        raise ValueError("one host buffer of each kind per step")
+    arrs = [_host_ptrs(x) for x in (q_host, k_host, v_host, W_host, out_host)]
+    cp, keep = _host_i32(cu_seqlens_host)
+    _check("iamap_prefill_steps_host", _lib.iamap_prefill_steps_host(
+        steps, *[ctypes.cast(a, ctypes.c_void_p) for a in arrs], _ptr(cu_seqlens), cp, num_seqs,
+        n, H_s, d, H_r, H_kv, d_v, B, tau, bias_window, bias_value, _ptr(lse), _ptr(mass),
+        _ptr(headmask_dense), _ptr(row_ptr), _ptr(col_idx), _ptr(headmask), _ptr(val_off),
+        _ptr(counts), _ptr(vals), vals_capacity_tiles, _ptr(io), io.numel() * io.element_size(),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    del keep, arrs
+
+
+def iamap_chunk_plan(cu_q_host, cu_k_host, starts_host, num_seqs, B):
+    qp, kq = _host_i32(cu_q_host)
+    kp, kk = _host_i32(cu_k_host)
+    sp, ks = _host_i32(starts_host)
+    nrb, ncb, mx = _I64(0), _I64(0), ctypes.c_int32(0)
+    _check("iamap_chunk_plan", _lib.iamap_chunk_plan(qp, kp, sp, num_seqs, B, ctypes.byref(nrb),
+                                                     ctypes.byref(ncb), ctypes.byref(mx)))
+    del kq, kk, ks
+    return nrb.value, ncb.value, mx.value
+
+
+def iamap_compress_chunk(q, k, cu_q, cu_k, starts, cu_q_host, cu_k_host, starts_host, num_seqs,
+                         n_q, n_k, H_s, d, B, tau, bias_window, bias_value, v_s, d_vs, o_s, lse,
+                         mass, headmask_dense, row_ptr, col_idx, headmask, val_off, counts, vals,
+                         vals_capacity_tiles, ws, stream=None):
+    qp, kq = _host_i32(cu_q_host)
+    kp, kk = _host_i32(cu_k_host)
+    sp, ks = _host_i32(starts_host)
+    _check("iamap_compress_chunk", _lib.iamap_compress_chunk(
+        _ptr(q), _ptr(k), _ptr(cu_q), _ptr(cu_k), _ptr(starts), qp, kp, sp, num_seqs, n_q, n_k,
+        H_s, d, B, tau, bias_window, bias_value, _ptr(v_s), d_vs, _ptr(o_s), _ptr(lse),
+        _ptr(mass), _ptr(headmask_dense), _ptr(row_ptr), _ptr(col_idx), _ptr(headmask),
+        _ptr(val_off), _ptr(counts), _ptr(vals), vals_capacity_tiles, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del kq, kk, ks
+
+
+def iamap_mapped_av_chunk(cu_q, cu_k, starts, cu_q_host, cu_k_host, starts_host, num_seqs, n_q,
+                          n_k, B, H_s, row_ptr, col_idx, headmask, val_off, vals,
+                          vals_capacity_tiles, W, H_r, H_kv, v, d_v, out, ws, stream=None):
+    qp, kq = _host_i32(cu_q_host)
+    kp, kk = _host_i32(cu_k_host)
+    sp, ks = _host_i32(starts_host)
+    _check("iamap_mapped_av_chunk", _lib.iamap_mapped_av_chunk(
+        _ptr(cu_q), _ptr(cu_k), _ptr(starts), qp, kp, sp, num_seqs, n_q, n_k, B, H_s,
+        _ptr(row_ptr), _ptr(col_idx), _ptr(headmask), _ptr(val_off), _ptr(vals),
+        vals_capacity_tiles, _ptr(W), H_r, H_kv, _ptr(v), d_v, _ptr(out), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del kq, kk, ks
 
 
 def iamap_mapped_av_paged_workspace_bytes(batch, H_r, d_v, max_ctx, page_size) -> int:

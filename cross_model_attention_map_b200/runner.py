@@ -61,6 +61,93 @@ class PrefillLayer:
         self.compress(q, k, stream)
         return self.mapped_av(W, v, stream, out)
 
+    def compress_with_output(self, q, k, v_s, o_s, stream=None):
+        """compress plus the sender's own attention output o_s [n, H_s, d_vs] from its values
+        v_s [n, H_s, d_vs] (same pass over the keys)."""
+        b = self.bufs
+        C.iamap_compress_with_output(q, k, self.cu, self.cu_host, self.num_seqs, self.n,
+                                     self.H_s, self.d, self.B, self.tau, self.bias_window,
+                                     self.bias_value, v_s, int(v_s.shape[2]), o_s, b["lse"],
+                                     b["mass"], b["headmask_dense"], b["row_ptr"], b["col_idx"],
+                                     b["headmask"], b["val_off"], b["counts"], self.vals,
+                                     self.capacity, self.ws, stream)
+        return o_s
+
+    def counts(self):
+        """(nnz_blocks, nnz_tiles) -- synchronises."""
+        c = self.bufs["counts"].cpu()
+        return int(c[0]), int(c[1])
+
+
+class ChunkPrefillLayer:
+    """Buffers of one chunked-prefill step of a mapped layer pair: the query rows
+    [starts[s], ends[s]) of every sequence s against its keys [0, ends[s]) (earlier chunks'
+    keys and values cached). starts[s] is a multiple of B. Optionally (d_vs given) the sender's
+    own attention output of the chunk rows is produced with the map.
+
+        compress(q, k, v_s=None) -> lse, masses, BSR map of the chunk rows (+ o_s)
+        mapped_av(W, v)          -> out [n_q, H_r, d_v]
+
+    q holds the chunk rows packed by cu_q; k, v (and v_s) hold rows [0, ends[s]) packed by cu_k.
+    """
+
+    def __init__(self, starts, ends, H_s, d, H_r, d_v, tau, bias_window=0, bias_value=0.0, B=64,
+                 capacity_tiles=None, device="cuda", H_kv=None, d_vs=None):
+        self.starts = [int(x) for x in starts]
+        self.ends = [int(x) for x in ends]
+        self.num_seqs = len(self.starts)
+        cu_q, cu_k = [0], [0]
+        for c0, e in zip(self.starts, self.ends):
+            cu_q.append(cu_q[-1] + e - c0)
+            cu_k.append(cu_k[-1] + e)
+        self.cu_q_host = torch.tensor(cu_q, dtype=torch.int32)
+        self.cu_k_host = torch.tensor(cu_k, dtype=torch.int32)
+        self.starts_host = torch.tensor(self.starts, dtype=torch.int32)
+        self.cu_q = self.cu_q_host.to(device)
+        self.cu_k = self.cu_k_host.to(device)
+        self.starts_dev = self.starts_host.to(device)
+        self.n_q, self.n_k = cu_q[-1], cu_k[-1]
+        self.H_s, self.d, self.H_r, self.d_v, self.B = H_s, d, H_r, d_v, B
+        self.H_kv = H_r if H_kv is None else int(H_kv)
+        self.tau, self.bias_window, self.bias_value = float(tau), int(bias_window), float(bias_value)
+        self.nrb, self.ncb, self.max_nb = C.iamap_chunk_plan(self.cu_q_host, self.cu_k_host,
+                                                             self.starts_host, self.num_seqs, B)
+        self.bufs = C.alloc_compress_outputs(self.n_q, H_s, self.nrb, self.ncb, device)
+        cap = H_s * self.ncb if capacity_tiles is None else int(capacity_tiles)
+        self.capacity = cap
+        self.vals = torch.empty(max(cap, 1), B, B, dtype=torch.bfloat16, device=device)
+        self.ws = C.alloc_workspace(C.iamap_compress_workspace_bytes(self.num_seqs, self.nrb),
+                                    device)
+        self.out = torch.empty(self.n_q, H_r, d_v, dtype=torch.float32, device=device)
+        self.d_vs = None if d_vs is None else int(d_vs)
+        self.o_s = (None if d_vs is None else
+                    torch.empty(self.n_q, H_s, self.d_vs, dtype=torch.float32, device=device))
+
+    def compress(self, q, k, v_s=None, stream=None):
+        b = self.bufs
+        C.iamap_compress_chunk(q, k, self.cu_q, self.cu_k, self.starts_dev, self.cu_q_host,
+                               self.cu_k_host, self.starts_host, self.num_seqs, self.n_q,
+                               self.n_k, self.H_s, self.d, self.B, self.tau, self.bias_window,
+                               self.bias_value, v_s, self.d_vs or 0,
+                               self.o_s if v_s is not None else None, b["lse"], b["mass"],
+                               b["headmask_dense"], b["row_ptr"], b["col_idx"], b["headmask"],
+                               b["val_off"], b["counts"], self.vals, self.capacity, self.ws,
+                               stream)
+
+    def mapped_av(self, W, v, stream=None, out=None):
+        b = self.bufs
+        out = self.out if out is None else out
+        C.iamap_mapped_av_chunk(self.cu_q, self.cu_k, self.starts_dev, self.cu_q_host,
+                                self.cu_k_host, self.starts_host, self.num_seqs, self.n_q,
+                                self.n_k, self.B, self.H_s, b["row_ptr"], b["col_idx"],
+                                b["headmask"], b["val_off"], self.vals, self.capacity, W,
+                                self.H_r, self.H_kv, v, self.d_v, out, self.ws, stream)
+        return out
+
+    def step(self, q, k, W, v, v_s=None, stream=None, out=None):
+        self.compress(q, k, v_s, stream)
+        return self.mapped_av(W, v, stream, out)
+
     def counts(self):
         """(nnz_blocks, nnz_tiles) -- synchronises."""
         c = self.bufs["counts"].cpu()
@@ -217,71 +304,40 @@ def gather_head_mapping(local_argmax, L_l, H_large, group=None):
 
 
 class HostPrefillPipeline:
-    """Prefill steps of one PrefillLayer on host-resident (pinned) inputs, with the upload of the
-    next step's q, k, v, W and the read-back of the previous step's output overlapping the current
-    step's kernels: two device sets of inputs and outputs, one upload and one download stream,
-    the kernels in order on the compute stream. Every step still moves its own inputs in and its
-    own output out."""
+    """Prefill steps of one PrefillLayer on host-resident (pinned) inputs through the library's
+    own host-buffer entry point (iamap_prefill_steps_host): every step uploads its q, k, v, W and
+    reads its output back, and the upload of the next step and the read-back of the previous one
+    overlap the current step's kernels (two device sets of inputs and outputs in `io`; the
+    library's upload and download streams, ordered by events against the compute stream)."""
 
     def __init__(self, layer, device="cuda"):
         self.layer = layer
-        self.up = torch.cuda.Stream(device)
-        self.down = torch.cuda.Stream(device)
-        dev = torch.device(device)
-        n, H_s, d, H_r, H_kv, d_v = layer.n, layer.H_s, layer.d, layer.H_r, layer.H_kv, layer.d_v
-        self.sets = [dict(q=torch.empty(n, H_s, d, dtype=torch.bfloat16, device=dev),
-                          k=torch.empty(n, H_s, d, dtype=torch.bfloat16, device=dev),
-                          v=torch.empty(n, H_kv, d_v, dtype=torch.bfloat16, device=dev),
-                          W=torch.empty(H_r, H_s, dtype=torch.float32, device=dev),
-                          out=torch.empty(n, H_r, d_v, dtype=torch.float32, device=dev))
-                     for _ in range(2)]
-        self.uploaded = [torch.cuda.Event() for _ in range(2)]
-        self.computed = [torch.cuda.Event() for _ in range(2)]
-        self.downloaded = [torch.cuda.Event() for _ in range(2)]
+        L = layer
+        self.io = C.alloc_workspace(C.iamap_prefill_io_bytes(L.n, L.H_s, L.d, L.H_r, L.H_kv,
+                                                             L.d_v), device)
 
     def bytes_per_step(self):
         """(host-to-device, device-to-host) bytes of one step."""
-        st = self.sets[0]
-        h2d = sum(st[x].numel() * st[x].element_size() for x in ("q", "k", "v", "W"))
-        return h2d, st["out"].numel() * st["out"].element_size()
+        L = self.layer
+        h2d = 2 * 2 * L.n * L.H_s * L.d + 2 * L.n * L.H_kv * L.d_v + 4 * L.H_r * L.H_s
+        return h2d, 4 * L.n * L.H_r * L.d_v
 
-    def run(self, host_inputs, host_outputs, stream=None, start_event=None):
+    def run(self, host_inputs, host_outputs, stream=None):
         """host_inputs[i] = (q, k, v, W) pinned CPU tensors of step i; host_outputs[i] the pinned
         CPU tensor receiving its output (entries may repeat: a buffer is written in step order).
-        Enqueues every step and returns the event recorded on `stream` after the last read-back.
-        start_event (recorded on `stream` by the caller) gates the first upload."""
+        Enqueues every step (the first upload follows everything enqueued on `stream` before)
+        and returns the event recorded on `stream` after the last read-back."""
         comp = torch.cuda.current_stream() if stream is None else stream
-        n = len(host_inputs)
-
-        def upload(i):
-            s = i % 2
-            with torch.cuda.stream(self.up):
-                if i == 0 and start_event is not None:
-                    self.up.wait_event(start_event)
-                if i >= 2:
-                    self.up.wait_event(self.computed[s])    # step i - 2 has read set s
-                for name, h in zip(("q", "k", "v", "W"), host_inputs[i]):
-                    self.sets[s][name].copy_(h, non_blocking=True)
-                self.uploaded[s].record(self.up)
-
-        if n:
-            upload(0)
-        for i in range(n):
-            s = i % 2
-            st = self.sets[s]
-            if i + 1 < n:
-                upload(i + 1)
-            comp.wait_event(self.uploaded[s])
-            if i >= 2:
-                comp.wait_event(self.downloaded[s])          # step i - 2's output was read back
-            self.layer.step(st["q"], st["k"], st["W"], st["v"], comp, out=st["out"])
-            self.computed[s].record(comp)
-            with torch.cuda.stream(self.down):
-                self.down.wait_event(self.computed[s])
-                host_outputs[i].copy_(st["out"], non_blocking=True)
-                self.downloaded[s].record(self.down)
+        L = self.layer
+        b = L.bufs
+        if host_inputs:
+            qs, ks, vs, Ws = (list(x) for x in zip(*host_inputs))
+            C.iamap_prefill_steps_host(qs, ks, vs, Ws, list(host_outputs), L.cu, L.cu_host,
+                                       L.num_seqs, L.n, L.H_s, L.d, L.H_r, L.H_kv, L.d_v, L.B,
+                                       L.tau, L.bias_window, L.bias_value, b["lse"], b["mass"],
+                                       b["headmask_dense"], b["row_ptr"], b["col_idx"],
+                                       b["headmask"], b["val_off"], b["counts"], L.vals,
+                                       L.capacity, self.io, L.ws, comp)
         done = torch.cuda.Event(enable_timing=True)
-        if n:
-            comp.wait_event(self.downloaded[(n - 1) % 2])
         done.record(comp)
         return done

@@ -23,6 +23,12 @@
  *                (section 3).
  *   *_gqa        mapped_av / mapped_av_paged with grouped receiver values: H_kv value heads,
  *                receiver head r reads value head r / (H_r / H_kv).
+ *   prefill_steps_host  end-to-end steps on host-resident inputs, the copies overlapping the
+ *                kernels of neighbouring steps.
+ *   compress_with_output, *_chunk  the sender's own attention output fused into compress, and
+ *                the chunked-prefill form of compress and mapped_av (query rows of a chunk
+ *                against all earlier keys). (MapFlow news page: the sender runs its own
+ *                attention; the fused kernel works with chunked prefill.)
  *   prefix index the prefix-hash index of stored map blocks: chained FNV-1a-64 keys of every full
  *                block of a prompt, insert of (key, location) pairs into a device hash table,
  *                lookup of a prompt's blocks and of its longest cached prefix. (MapFlow news
@@ -189,6 +195,109 @@ int iamap_mapped_av_gqa(const int32_t* cu_seqlens, const int32_t* cu_seqlens_hos
                         int64_t vals_capacity_tiles, const float* W, int H_r, int H_kv,
                         const void* v, int d_v, float* out, void* ws, size_t ws_bytes,
                         void* stream);
+
+/*
+ * Compress with the sender's own attention output. As iamap_compress (stages 1 and 2), and in
+ * the same pass over the keys the sender output O_s[i, h] = sum_{j <= i} p_h(i, j) V_s[j, h]
+ * with the probabilities p of the map before any block is dropped (the bf16-rounded values the
+ * stored tiles hold). The sender runs its own attention while its map is recorded for the
+ * receiver ("PKU MapFlow" news page, the paragraphs on the attention map as the shared state).
+ *   v_s   bf16 [n, H_s, d_vs]  the sender's values, d_vs 64 or 128, 16-byte aligned
+ *   o_s   fp32 [n, H_s, d_vs]  written in full
+ * Sequences may hold at most 256 blocks of 64 (IAMAP_ERR_UNSUPPORTED otherwise). The workspace
+ * is iamap_compress_workspace_bytes(num_seqs, num_rowblocks). Other arguments and outputs as
+ * iamap_compress.
+ */
+int iamap_compress_with_output(const void* q, const void* k, const int32_t* cu_seqlens,
+                               const int32_t* cu_seqlens_host, int num_seqs, int64_t n, int H_s,
+                               int d, int B, float tau, int bias_window, float bias_value,
+                               const void* v_s, int d_vs, float* o_s, float* lse, float* mass,
+                               uint64_t* headmask_dense, int32_t* row_ptr, int32_t* col_idx,
+                               uint64_t* headmask, int64_t* val_off, int64_t* counts, void* vals,
+                               int64_t vals_capacity_tiles, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/*
+ * Chunked prefill ("PKU MapFlow" news page, the paragraph on the vLLM integration: the fused
+ * kernel works with chunked prefill). Sequence s of a batch has keys [0, e_s), e_s =
+ * cu_k[s+1] - cu_k[s], and a chunk of query rows [starts[s], e_s); starts[s] is a multiple of
+ * B (0 = the whole sequence). The chunk attends to all keys [0, e_s) with absolute positions in
+ * the causal mask and the local bias, so its results equal the whole-sequence results of those
+ * rows. Its row blocks are the sequence's own row blocks I = starts[s]/B .. ceil(e_s/B) - 1.
+ *   q        bf16 [n_q, H_s, d]    the chunks' query rows, packed by cu_q (int32 [S+1],
+ *                                  cu_q[s+1] - cu_q[s] = e_s - starts[s])
+ *   k        bf16 [n_k, H_s, d]    the keys [0, e_s) of every sequence, packed by cu_k
+ *   starts   int32 [S]             chunk starts (device); *_host: the same values on the host
+ * Chunk layouts: the listed row blocks are the chunks' row blocks, sequence-major, and the causal
+ * blocks (I, J <= I) of those row blocks; iamap_chunk_plan reports their numbers. lse is
+ * [H_s, n_q] (packed query rows), mass [H_s, num_causal_blocks], the BSR index has
+ * num_rowblocks + 1 row pointers; col_idx stays the sequence-local column block J.
+ */
+int iamap_chunk_plan(const int32_t* cu_q_host, const int32_t* cu_k_host,
+                     const int32_t* starts_host, int num_seqs, int B, int64_t* num_rowblocks,
+                     int64_t* num_causal_blocks, int32_t* max_blocks_per_seq);
+
+/*
+ * Compress of a batch of chunks (stages 1 and 2 in one call, as iamap_compress), optionally with
+ * the sender output of the chunk rows: v_s bf16 [n_k, H_s, d_vs] packed like k, o_s fp32
+ * [n_q, H_s, d_vs] (both NULL: no sender output). Sequences may hold at most 256 blocks of 64.
+ * Workspace: iamap_compress_workspace_bytes(num_seqs, num_rowblocks of the chunk plan).
+ * Errors as iamap_compress; IAMAP_ERR_INVALID_ARG if a start is not a multiple of B or a chunk
+ * does not end at its key length.
+ */
+int iamap_compress_chunk(const void* q, const void* k, const int32_t* cu_q, const int32_t* cu_k,
+                         const int32_t* starts, const int32_t* cu_q_host,
+                         const int32_t* cu_k_host, const int32_t* starts_host, int num_seqs,
+                         int64_t n_q, int64_t n_k, int H_s, int d, int B, float tau,
+                         int bias_window, float bias_value, const void* v_s, int d_vs,
+                         float* o_s, float* lse, float* mass, uint64_t* headmask_dense,
+                         int32_t* row_ptr, int32_t* col_idx, uint64_t* headmask,
+                         int64_t* val_off, int64_t* counts, void* vals,
+                         int64_t vals_capacity_tiles, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * mapped_av of a batch of chunks: out fp32 [n_q, H_r, d_v] (the chunk rows, packed by cu_q) from
+ * the chunk BSR map of iamap_compress_chunk and the receiver's values v bf16 [n_k, H_kv, d_v]
+ * packed like the keys (grouped values as iamap_mapped_av_gqa; H_kv = H_r for one value head per
+ * receiver head).
+ */
+int iamap_mapped_av_chunk(const int32_t* cu_q, const int32_t* cu_k, const int32_t* starts,
+                          const int32_t* cu_q_host, const int32_t* cu_k_host,
+                          const int32_t* starts_host, int num_seqs, int64_t n_q, int64_t n_k,
+                          int B, int H_s, const int32_t* row_ptr, const int32_t* col_idx,
+                          const uint64_t* headmask, const int64_t* val_off, const void* vals,
+                          int64_t vals_capacity_tiles, const float* W, int H_r, int H_kv,
+                          const void* v, int d_v, float* out, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/*
+ * End-to-end prefill steps from host memory. For each step i < steps: upload q_host[i],
+ * k_host[i] (bf16 [n, H_s, d]), v_host[i] (bf16 [n, H_kv, d_v]) and W_host[i] (fp32 [H_r, H_s]),
+ * run iamap_compress and iamap_mapped_av_gqa on them, and read the output back into out_host[i]
+ * (fp32 [n, H_r, d_v]). The host buffers should be pinned (page-locked): pageable memory works
+ * but its copies do not overlap the kernels.
+ *   io    device buffer of iamap_prefill_io_bytes bytes, 256-byte aligned: two sets of device
+ *         inputs and outputs, so that the upload of step i + 1 and the read-back of step i - 1
+ *         overlap the kernels of step i. The copies run on an upload and a download stream that
+ *         the library creates once per device; events order them against `stream`, on which the
+ *         kernels run. One cudaMemcpyAsync per copy.
+ *   lse .. vals_capacity_tiles, ws   the compress buffers and workspace, as for iamap_compress
+ *         (reused by every step).
+ * Enqueues everything and returns; `stream` then waits for the last read-back, so an event
+ * recorded or a synchronisation made on `stream` after the call covers every step. Errors as
+ * iamap_compress / iamap_mapped_av_gqa, and IAMAP_ERR_WORKSPACE if io is too small.
+ */
+size_t iamap_prefill_io_bytes(int64_t n, int H_s, int d, int H_r, int H_kv, int d_v);
+int iamap_prefill_steps_host(int steps, const void* const* q_host, const void* const* k_host,
+                             const void* const* v_host, const float* const* W_host,
+                             float* const* out_host, const int32_t* cu_seqlens,
+                             const int32_t* cu_seqlens_host, int num_seqs, int64_t n, int H_s,
+                             int d, int H_r, int H_kv, int d_v, int B, float tau, int bias_window,
+                             float bias_value, float* lse, float* mass, uint64_t* headmask_dense,
+                             int32_t* row_ptr, int32_t* col_idx, uint64_t* headmask,
+                             int64_t* val_off, int64_t* counts, void* vals,
+                             int64_t vals_capacity_tiles, void* io, size_t io_bytes, void* ws,
+                             size_t ws_bytes, void* stream);
 
 /*
  * Decode step on a mapped layer: one query row per sequence b.

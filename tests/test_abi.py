@@ -190,3 +190,43 @@ int main(void) {
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
     assert out.stdout.startswith("ok 6 12 4 4")
+
+
+def test_chunk_plan_counts_and_checks(lib):
+    """Chunk plan on the host: only the chunks' row blocks and causal blocks are counted; starts
+    that are not multiples of B, or chunks that do not end at their key length, are refused."""
+    # sequence 0: keys 228 (4 blocks), chunk from 128 (blocks 2, 3); sequence 1: keys 192
+    # (3 blocks), chunk from 128 (block 2)
+    assert lib.iamap_chunk_plan([0, 100, 164], [0, 228, 420], [128, 128], 2, 64) == (3, 7 + 3, 4)
+    # whole sequences as chunks: the plan of the sequences themselves
+    assert lib.iamap_chunk_plan([0, 4096, 12288], [0, 4096, 12288], [0, 0], 2, 64) == \
+        lib.iamap_plan([0, 4096, 12288], 2, 64)
+    # a chunk at the end of a sequence that holds no rows
+    assert lib.iamap_chunk_plan([0, 0], [0, 128], [128], 1, 64) == (0, 0, 2)
+    with pytest.raises(lib.IamapError) as e:
+        lib.iamap_chunk_plan([0, 200], [0, 300], [100], 1, 64)       # 100 is not a multiple of 64
+    assert e.value.code == -1 and "multiple" in lib.iamap_last_error()
+    with pytest.raises(lib.IamapError) as e:
+        lib.iamap_chunk_plan([0, 100], [0, 300], [128], 1, 64)       # ends at 228, keys 300
+    assert e.value.code == -1
+
+
+def test_host_validation_of_chunk_and_sender_output(lib):
+    """The chunk and sender-output entry points refuse bad arguments before any device work."""
+    raw = lib._lib
+    fake = 256   # never dereferenced: every call below fails validation first
+    # d_vs must be 64 or 128
+    rc = raw.iamap_compress_with_output(fake, fake, fake, None, 1, 64, 4, 64, 64, 0.9, 0, 0.0,
+                                        fake, 96, fake, fake, fake, fake, fake, fake, fake, fake,
+                                        fake, fake, 1, fake, 0, None)
+    assert rc == -2 and "d_vs" in lib.iamap_last_error()
+    # v_s without o_s
+    rc = raw.iamap_compress_chunk(fake, fake, fake, fake, fake, None, None, None, 1, 64, 64, 4, 64,
+                                  64, 0.9, 0, 0.0, fake, 64, None, fake, fake, fake, fake, fake,
+                                  fake, fake, fake, fake, 1, fake, 0, None)
+    assert rc == -1 and "together" in lib.iamap_last_error()
+    # grouped values must divide the receiver heads
+    rc = raw.iamap_mapped_av_chunk(fake, fake, fake, None, None, None, 1, 64, 64, 64, 4, fake,
+                                   fake, fake, fake, fake, 1, fake, 8, 3, fake, 64, fake, fake, 0,
+                                   None)
+    assert rc == -1 and "divide" in lib.iamap_last_error()
