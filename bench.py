@@ -45,12 +45,19 @@ CONFIG_TEXT = {
     "varlen40k": ("varlen40k: 4 packed causal sequences 4096/8192/12288/16384 (40960 tokens), "
                   "sender H_s=40 d=128, receiver H_r=32 d_v=128, B=64, tau=0.9, sink; "
                   "compress + mapped_av"),
+    "varlen40k_sender": ("varlen40k_sender: the varlen40k workload with the sender's own "
+                         "attention output (values d_vs=128) fused into compress; compress + "
+                         "sender output + mapped_av"),
     "prefill8k": ("prefill8k: 1 causal sequence n=8192, H_s=32 d=128, H_r=24 d_v=128, B=64, "
                   "tau=0.95, sink, local bias +2.0 on |i-j|<128; compress + mapped_av"),
     "tiny": "tiny: n=512, H_s=8 d=64, H_r=4 d_v=64, B=64, tau=0.95, sink; compress + mapped_av",
     "headmatch": ("headmatch: n=1024, small 24 layers x 14 heads d=64, large 8 layers x 64 heads "
                   "d=128, planted noisy copies; head_match"),
-    "decode": ("decode: batch 4, q_len 1, context 8704, sender 14 heads, receiver 64 heads "
+    "headmatch8k": ("headmatch8k: the headmatch calibration at prompt length n=8192 (small 24 "
+                    "layers x 14 heads d=64, large 8 layers x 64 heads d=128, planted noisy "
+                    "copies); head_match"),
+    "decode": ("decode: batch 4, q_len 1, context 8704, sender 14 heads d=64 (its softmax rows "
+               "over its paged keys, computed before the timed region), receiver 64 heads "
                "d_v=128, one-hot W, 16-token pages; mapped_av_paged"),
     "prefixindex": ("prefixindex: publish the 4 varlen prompts (40960 tokens, 640 blocks of 64) "
                     "into an empty 4096-slot prefix-hash index, then look up 16 prompts "
@@ -259,30 +266,62 @@ def max_over_ranks(x, world):
 # CPU baseline: the oracle on a bounded sample
 # ------------------------------------------------------------------------------------------------
 
-def oracle_sample_prefill(wl, budget_s=20.0, seed=0):
-    """Oracle compress + mapped_av on random row blocks (all sender and receiver heads) until the
-    budget is used. Returns (tokens/s, rows, seconds, sample text)."""
+def systematic_rowblocks(wl, count=5):
+    """A fixed sample of `count` row blocks of the workload: every (nrb // count)-th row block of
+    the sequence-major enumeration, from the middle of the first stride. Row blocks later in a
+    sequence cost more (more keys), and an evenly spaced sample follows that mix."""
     import oracle as O
     lay = O.causal_layout(wl.seqlens, wl.B)
-    rng = np.random.default_rng(seed)
     blocks = [(s, I) for s in range(len(wl.seqlens)) for I in range(lay.nb[s])]
-    order = rng.permutation(len(blocks))
+    count = max(1, min(count, len(blocks)))
+    stride = len(blocks) // count
+    return [blocks[stride // 2 + j * stride] for j in range(count)]
+
+
+def oracle_rowblock(wl, s, I):
+    """Oracle compress (all sender heads) + mapped_av rows of one row block: the per-head stats
+    (kept sets, near marks) and the number of query rows."""
+    import oracle as O
+    st = {h: O.rowblock_stats(wl.q, wl.k, wl.cu_seqlens, s, h, I, wl.B, wl.tau,
+                              wl.bias_window, wl.bias_value) for h in range(wl.H_s)}
+    O.mapped_av_rows(wl, s, I, lambda h: st[h].kept, lambda h: st[h])
+    return st, st[0].R
+
+
+def oracle_sample_prefill(wl, blocks):
+    """Oracle compress + mapped_av on the given row blocks (all sender and receiver heads).
+    Returns (tokens/s, rows, seconds, per-block stats, sample text)."""
     rows = 0
+    stats = []
     t0 = time.perf_counter()
-    done = 0
-    for idx in order:
-        s, I = blocks[idx]
-        st = {h: O.rowblock_stats(wl.q, wl.k, wl.cu_seqlens, s, h, I, wl.B, wl.tau,
-                                  wl.bias_window, wl.bias_value) for h in range(wl.H_s)}
-        O.mapped_av_rows(wl, s, I, lambda h: st[h].kept, lambda h: st[h])
-        rows += st[0].R
-        done += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
+    for s, I in blocks:
+        st, R = oracle_rowblock(wl, s, I)
+        rows += R
+        stats.append((s, I, st))
     dt = time.perf_counter() - t0
-    text = ("%d uniformly drawn row blocks of %d (%d query rows, all %d sender and %d receiver "
-            "heads): float64 compress + mapped_av" % (done, len(blocks), rows, wl.H_s, wl.H_r))
-    return rows / dt, rows, dt, text
+    text = ("%d row blocks %s (sequence, row block) of %d sequences (%d query rows, all %d sender "
+            "and %d receiver heads): float64 compress + mapped_av"
+            % (len(blocks), [tuple(b) for b in blocks], len(wl.seqlens), rows, wl.H_s, wl.H_r))
+    return rows / dt, rows, dt, stats, text
+
+
+def kept_set_check(wl, kept_gpu, stats):
+    """Kept sets of the GPU against the oracle's on the sampled row blocks: blocks compared,
+    near-threshold blocks, flips (all near-threshold) and mismatches outside them."""
+    import oracle as O
+    lay = O.causal_layout(wl.seqlens, wl.B)
+    blocks = near = flips = bad = 0
+    for s, I, st in stats:
+        c0 = lay.cb(s, I, 0)
+        for h in range(wl.H_s):
+            g = kept_gpu[h, c0:c0 + I + 1]
+            diff = g != st[h].kept
+            blocks += I + 1
+            near += int(st[h].near.sum())
+            flips += int((diff & st[h].near).sum())
+            bad += int((diff & ~st[h].near).sum())
+    return {"sampled_rowblocks": len(stats), "blocks": blocks, "near_threshold": near,
+            "flips": flips, "mismatches_outside_near": bad}
 
 
 def cores():
@@ -301,6 +340,32 @@ def bf16_dev(bits, device):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
 
 
+def base_config(name):
+    """The prefill workload a bench configuration runs on (a "_sender" configuration adds the
+    sender's own output to its base workload)."""
+    return name[:-len("_sender")] if name.endswith("_sender") else name
+
+
+def split_by_sequence(wl_full, world, rank):
+    """This rank's sub-batch of a packed prefill batch split by sequence (longest first by
+    causal blocks, runner.shard_sequences): (workload of its sequences, their indices)."""
+    from synth import select_sequences
+    from cross_model_attention_map_b200.runner import shard_sequences
+    mine = shard_sequences(wl_full.seqlens, world, wl_full.B)[rank]
+    return select_sequences(wl_full, mine), mine
+
+
+def idle_rank(args, world, tokens_total):
+    """A rank that holds no sequence of a split batch: it takes the same barriers and max
+    reductions as the others (with zero time), and reports nothing."""
+    for _ in range(2):
+        barrier(world)
+    ms = max_over_ranks(0.0, world)
+    barrier(world)
+    e2e_ms = max_over_ranks(0.0, world)
+    return {"idle": True, "ms": ms, "e2e_ms": e2e_ms, "tokens_total": tokens_total}
+
+
 def bench_prefill(args, world, rank, local, peaks):
     import torch
     from synth import prefill_config
@@ -308,7 +373,18 @@ def bench_prefill(args, world, rank, local, peaks):
     from cross_model_attention_map_b200.runner import PrefillLayer
 
     dev = torch.device("cuda", local)
-    wl = prefill_config(args.config, seed=rank)
+    if args.split == "seq":
+        # one packed batch split by sequence over the ranks (strong scaling, no collective on
+        # the path)
+        wl_full = prefill_config(base_config(args.config), seed=0)
+        wl, mine = split_by_sequence(wl_full, world, rank)
+        tokens_total = wl_full.n
+    else:
+        wl = prefill_config(base_config(args.config), seed=rank)
+        mine = list(range(len(wl.seqlens)))
+        tokens_total = wl.n * world
+    if not mine:
+        return idle_rank(args, world, tokens_total), wl
     q, k, v = bf16_dev(wl.q, dev), bf16_dev(wl.k, dev), bf16_dev(wl.v, dev)
     W = torch.from_numpy(wl.W).to(dev)
     layer = PrefillLayer(wl.seqlens, wl.H_s, wl.d, wl.H_r, wl.d_v, wl.tau, wl.bias_window,
@@ -322,7 +398,20 @@ def bench_prefill(args, world, rank, local, peaks):
                                b["mass"], b["headmask_dense"], b["row_ptr"], b["col_idx"],
                                b["headmask"], b["val_off"], b["counts"], layer.ws, stream)
 
+    sender = args.config.endswith("_sender")
+    if sender:
+        from synth import make_sender_values
+        v_s = bf16_dev(make_sender_values(wl), dev)
+        o_s = torch.empty(wl.n, wl.H_s, wl.d, dtype=torch.float32, device=dev)
+
     def extract():
+        if sender:
+            C.iamap_compress_extract_with_output(
+                q, k, layer.cu, layer.cu_host, layer.num_seqs, layer.n, wl.H_s, wl.d, wl.B,
+                wl.bias_window, wl.bias_value, v_s, wl.d, o_s, b["lse"], b["row_ptr"],
+                b["col_idx"], b["headmask"], b["val_off"], b["counts"], layer.vals,
+                layer.capacity, layer.ws, stream)
+            return
         C.iamap_compress_extract(q, k, layer.cu, layer.cu_host, layer.num_seqs, layer.n, wl.H_s,
                                  wl.d, wl.B, wl.bias_window, wl.bias_value, b["lse"],
                                  b["row_ptr"], b["col_idx"], b["headmask"], b["val_off"],
@@ -375,7 +464,6 @@ def bench_prefill(args, world, rank, local, peaks):
     assert C.iamap_device_status(stream) == 0
 
     n = layer.n
-    tokens_total = n * world
     value = tokens_total / (ms * 1e-3)
 
     # algorithmic work per launch
@@ -385,6 +473,8 @@ def bench_prefill(args, world, rank, local, peaks):
     av_bytes = (8192.0 * nnz_tiles + 20.0 * nnz_blocks + 4.0 * (layer.nrb + 1)
                 + 2.0 * n * wl.H_r * wl.d_v + 4.0 * n * wl.H_r * wl.d_v + 4.0 * wl.H_r * wl.H_s)
     extract_bytes = 8192.0 * nnz_tiles + 2.0 * 2 * n * wl.H_s * wl.d + 4.0 * n * wl.H_s
+    if sender:   # the sender's values read once, its output written once
+        extract_bytes += 2.0 * n * wl.H_s * wl.d + 4.0 * n * wl.H_s * wl.d
     kernels = {
         "compress_stats": {"ms": t_stats, "bound": "alu", "exps": exps,
                            "gex2_per_s": exps / (t_stats * 1e-3) / 1e9,
@@ -448,9 +538,13 @@ def bench_prefill(args, world, rank, local, peaks):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if args.split == "seq" else "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; the configuration's shapes and distributions)",
         "config": {"workload": CONFIG_TEXT[args.config], "tokens_per_gpu": n,
+                   "split": ("sequences %s of the packed batch on rank %d (longest first by "
+                             "causal blocks)" % (mine, rank)) if args.split == "seq"
+                            else "one whole batch per GPU",
                    "nnz_blocks": nnz_blocks, "nnz_tiles": nnz_tiles,
                    "kept_tile_density": round(nnz_tiles / (wl.H_s * layer.ncb), 4),
                    "l2": ("inputs larger than L2 (Q+K %.0f MB, BSR values %.1f GB); no flush"
@@ -458,7 +552,9 @@ def bench_prefill(args, world, rank, local, peaks):
                           if flush is None else
                           "inputs fit in L2 (%.1f MB): 256 MB buffer written between timed "
                           "steps, outside the step's events" % (step_bytes / 1e6)),
-                   "parallelism": "dp%d (independent batches per GPU, no collective)" % world},
+                   "parallelism": ("sequence split over %d GPUs (no collective)" % world
+                                   if args.split == "seq" else
+                                   "dp%d (independent batches per GPU, no collective)" % world)},
         "kernels": {kk: {x: (round(y, 4) if isinstance(y, float) else y) for x, y in kv.items()}
                     for kk, kv in kernels.items()},
         "roofline": roofline,
@@ -468,6 +564,9 @@ def bench_prefill(args, world, rank, local, peaks):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
     }
+    hm = layer.bufs["headmask_dense"].cpu().numpy().view(np.uint64)
+    line["_kept"] = ((hm[None, :] >> np.arange(wl.H_s, dtype=np.uint64)[:, None])
+                     & np.uint64(1)).astype(bool)
     return line, wl
 
 
@@ -481,11 +580,19 @@ def bench_decode(args, world, rank, local, peaks):
     dw = decode_config(seed=rank)
     st = DecodeStep(dw.batch, dw.H_s, dw.H_r, dw.d_v, dw.ctx_lens, dw.p_rows.shape[2],
                     dw.page_table.shape[1], dw.page_size, dw.v_pages.shape[0], device=dev)
-    p = torch.from_numpy(dw.p_rows).to(dev)
     W = torch.from_numpy(dw.W).to(dev)
     vp = bf16_dev(dw.v_pages, dev)
     pt = torch.from_numpy(dw.page_table).to(dev)
     stream = torch.cuda.current_stream()
+    # the sender rows: the small model's own softmax rows over its paged keys, computed by the
+    # library before the timed region (the small model runs its attention anyway)
+    max_ctx = int(dw.ctx_lens.max())
+    p = torch.empty(dw.batch, dw.H_s, max_ctx, dtype=torch.float32, device=dev)
+    rws = C.alloc_workspace(C.iamap_sender_rows_workspace_bytes(dw.batch, dw.H_s, max_ctx), dev)
+    C.iamap_sender_rows(bf16_dev(dw.q_s, dev), bf16_dev(dw.k_pages_s, dev),
+                        dw.k_pages_s.shape[0], pt, dw.page_table.shape[1], dw.page_size,
+                        st.ctx_lens, dw.ctx_lens, dw.batch, dw.H_s, dw.q_s.shape[2], p, max_ctx,
+                        rws, stream)
     for _ in range(args.warmup):
         st.run(p, W, vp, pt, stream)
     torch.cuda.synchronize()
@@ -529,7 +636,11 @@ def bench_headmatch(args, world, rank, local, peaks):
     from cross_model_attention_map_b200.runner import HeadMatch
 
     dev = torch.device("cuda", local)
-    hm = head_match_config(seed=rank)
+    if args.config == "headmatch8k":
+        from synth import make_head_match
+        hm = make_head_match(n=8192, seed=rank)
+    else:
+        hm = head_match_config(seed=rank)
     r = HeadMatch(hm.L_s, hm.H_small, hm.d_small, hm.L_l, hm.H_large, hm.d_large, hm.n,
                   want_sim=False, device=dev)
     qs, ks = bf16_dev(hm.q_small, dev), bf16_dev(hm.k_small, dev)
@@ -558,20 +669,23 @@ def bench_headmatch(args, world, rank, local, peaks):
     gram = 2.0 * NS * NL * pairs
     maps = 2.0 * pairs * (NS * hm.d_small + NL * hm.d_large)
     tf = (gram + maps) / (ms * 1e-3) / 1e12
+    planted = float((r.argmax.cpu().numpy().reshape(hm.L_l, hm.H_large) == hm.planted).mean())
     return {
-        "metric": "head_match calibrations/s (n=1024, 336 small x 512 large heads)",
+        "metric": "head_match calibrations/s (n=%d, 336 small x 512 large heads)" % hm.n,
         "value": round(world / (ms * 1e-3), 2), "unit": "calibrations/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": {"workload": CONFIG_TEXT["headmatch"],
+        "data": "synthetic", "config": {"workload": CONFIG_TEXT[args.config],
                                         "gram_K_padded": K,
+                                        "planted_mapping_recovered": planted,
                                         "l2": "inputs larger than L2 (Q, K of both models "
                                               "%.0f MB); no flush" % (2.0 * (
                                                   qs.numel() + ks.numel() + ql.numel()
                                                   + kl.numel()) / 1e6)},
         "roofline": {"kernel": "head_match (maps + gram)", "bound": "tensor",
                      "achieved": round(tf, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None},
+                     "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None,
+                     "flops": {"gram": gram, "maps_qk": maps}},
         "clocks": clocks, "gpu_launches": 5 * args.steps,
     }, hm
 
@@ -763,23 +877,32 @@ def reference_arm(args):
                           "no reference arm for this configuration"}))
         return
     wl = prefill_config(args.config)
-    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
-    for _ in range(args.warmup):
-        oracle_sample_prefill(wl, budget_s=budget, seed=99)
-    vals = []
-    text = ""
+    sample = systematic_rowblocks(wl)
+    for i in range(args.warmup):
+        oracle_rowblock(wl, *sample[i % len(sample)])
+    rows = 0
+    step_s = []
     for i in range(args.steps):
-        v, rows, dt, text = oracle_sample_prefill(wl, budget_s=budget, seed=i)
-        vals.append(v)
-    value = statistics.mean(vals)
-    ms = 1e3 * sum(wl.seqlens) / value
+        t0 = time.perf_counter()
+        _, R = oracle_rowblock(wl, *sample[i % len(sample)])
+        step_s.append(time.perf_counter() - t0)
+        rows += R
+    secs = sum(step_s)
+    value = rows / secs
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
-        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / args.steps, 2),
+        "ms_per_workload_extrapolated": round(1e3 * sum(wl.seqlens) / value, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": CONFIG_TEXT[args.config]},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores(),
-                         "kind": "oracle", "sample": text + " per step"},
+                         "kind": "oracle",
+                         "sample": "step i: row block i mod %d of the fixed sample %s (sequence, "
+                                   "row block), all %d sender and %d receiver heads; %d query "
+                                   "rows timed in %.1f s over %d steps"
+                                   % (len(sample), [tuple(b) for b in sample], wl.H_s, wl.H_r,
+                                      rows, secs, args.steps)},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }))
@@ -792,9 +915,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="varlen40k", choices=sorted(CONFIG_TEXT))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--cpu-budget", type=float, default=20.0,
-                    help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split", default="batch", choices=["batch", "seq"],
+                    help="multi-GPU prefill: one whole batch per GPU (weak scaling) or one packed "
+                         "batch split by sequence (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -807,7 +931,7 @@ def main():
 
     world, rank, local = dist_setup(args)
     peaks = load_peaks()
-    if args.config in ("varlen40k", "prefill8k", "tiny"):
+    if base_config(args.config) in ("varlen40k", "prefill8k", "tiny"):
         line, wl = bench_prefill(args, world, rank, local, peaks)
     elif args.config == "decode":
         line, wl = bench_decode(args, world, rank, local, peaks)
@@ -815,16 +939,22 @@ def main():
         line, wl = bench_prefixindex(args, world, rank, local, peaks)
     else:
         line, wl = bench_headmatch(args, world, rank, local, peaks)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config in (
+    kept_gpu = line.pop("_kept", None)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and base_config(args.config) in (
             "varlen40k", "prefill8k", "tiny"):
-        v, rows, dt, text = oracle_sample_prefill(wl, budget_s=args.cpu_budget)
+        v, rows, dt, stats, text = oracle_sample_prefill(wl, systematic_rowblocks(wl))
         line["cpu_baseline"] = {"value": round(v, 2), "unit": "tokens/s", "cores": cores(),
                                 "kind": "oracle", "sample": text + " in %.1f s" % dt}
+        line["kept_set_check"] = kept_set_check(wl, kept_gpu, stats)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "decode":
         v, dt = oracle_decode_step(wl)
         line["cpu_baseline"] = {"value": round(v, 3), "unit": "rows/s", "cores": cores(),
                                 "kind": "oracle",
                                 "sample": "one whole decode step (batch 4) in %.1f s" % dt}
+    if rank == 0 and world == 1 and args.config == "headmatch8k":
+        line["cpu_baseline"] = None
+        line["cpu_baseline_note"] = ("none: the float64 oracle would hold the 336 small heads' "
+                                     "flattened 8192 x 8192 maps (180 GB)")
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "headmatch":
         v, dt = oracle_headmatch_sample(wl)
         line["cpu_baseline"] = {"value": round(v, 4), "unit": "calibrations/s",

@@ -213,6 +213,68 @@ extern "C" int iamap_compress_with_output(
   return compress_on_tables(a, counts, vals, vals_capacity_tiles, st);
 }
 
+extern "C" int iamap_compress_extract_with_output(
+    const void* q, const void* k, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+    int num_seqs, int64_t n, int H_s, int d, int B, int bias_window, float bias_value,
+    const void* v_s, int d_vs, float* o_s, const float* lse, const int32_t* row_ptr,
+    const int32_t* col_idx, const uint64_t* headmask, const int64_t* val_off,
+    const int64_t* counts, void* vals, int64_t vals_capacity_tiles, void* ws, size_t ws_bytes,
+    void* stream) {
+  clear_error();
+  int rc = check_chunk_common(B, H_s, d);
+  if (rc) return rc;
+  if (!q || !k || !cu_seqlens || !lse || !row_ptr || !col_idx || !headmask || !val_off ||
+      !counts || (!vals && vals_capacity_tiles > 0))
+    return set_error(IAMAP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!v_s || !o_s) return set_error(IAMAP_ERR_INVALID_ARG, "v_s and o_s are required");
+  if (d_vs != 64 && d_vs != 128)
+    return set_error(IAMAP_ERR_UNSUPPORTED, "sender value dim d_vs must be 64 or 128");
+  if (vals_capacity_tiles < 0) return set_error(IAMAP_ERR_INVALID_ARG, "negative capacity");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v_s) || !aligned16(o_s) ||
+      (vals && !aligned16(vals)))
+    return set_error(IAMAP_ERR_INVALID_ARG, "q, k, v_s, o_s, vals must be 16-byte aligned");
+  DeviceContext* ctx = device_context();
+  if (!ctx) return IAMAP_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CompressArgs a;
+  rc = make_plan(cu_seqlens_host, num_seqs, B, n, &a.plan);
+  if (rc) return rc;
+  if (!compress_tc_supported(d, a.plan.max_nb))
+    return set_error(IAMAP_ERR_UNSUPPORTED, "the sender output needs sequences of at most 256 "
+                     "blocks (%d given)", a.plan.max_nb);
+  const size_t need = seq_tables_bytes(num_seqs, a.plan.num_rowblocks);
+  if (!ws || ws_bytes < need)
+    return set_error(IAMAP_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                     ws_bytes);
+  a.tab = carve_seq_tables(ws, num_seqs, a.plan.num_rowblocks);
+  if (a.plan.num_rowblocks > 0) {
+    rc = launch_build_tables(cu_seqlens, num_seqs, B, a.plan.max_nb, a.tab, st);
+    if (rc) return rc;
+  }
+  a.q = q;
+  a.k = k;
+  a.cu_seqlens = cu_seqlens;
+  a.num_seqs = num_seqs;
+  a.n = n;
+  a.H_s = H_s;
+  a.d = d;
+  a.bias_window = bias_window;
+  a.bias_value = bias_value;
+  a.lse_in = lse;
+  a.row_ptr_in = row_ptr;
+  a.col_idx_in = col_idx;
+  a.headmask_in = headmask;
+  a.val_off_in = val_off;
+  a.counts_in = counts;
+  a.vals = vals;
+  a.capacity = vals_capacity_tiles;
+  a.v_s = v_s;
+  a.d_vs = d_vs;
+  a.o_s = o_s;
+  a.status = ctx->status;
+  return compress_extract_impl(a, st);
+}
+
 extern "C" int iamap_mapped_av_chunk(
     const int32_t* cu_q, const int32_t* cu_k, const int32_t* starts, const int32_t* cu_q_host,
     const int32_t* cu_k_host, const int32_t* starts_host, int num_seqs, int64_t n_q, int64_t n_k,

@@ -810,7 +810,7 @@ static size_t extract_smem() {
   return 1024 + (size_t)(D / 64) * (kPanel128 + kXStages * kPanel64) +
          (OUT ? (size_t)kVStages * 2 * kPanel64 + 2 * 8 * 4096 : 8 * 4096) +
          sizeof(int64_t) * 2 * kMaxNb + sizeof(int) * 3 * kMaxNb +
-         8 * (OUT ? XO_NUM_BARS : X_NUM_BARS) + 16;
+         8 * (OUT ? (int)XO_NUM_BARS : (int)X_NUM_BARS) + 16;
 }
 
 }  // namespace tccomp

@@ -105,10 +105,6 @@ constexpr int kMaxNP = 12;       // sender-slice ring: as many slots as shared m
 // spread over several producer warps: four for the sender slices (chunks round-robin) and one
 // per receiver head for the V tiles (each a single 3-D box of both 64-dim halves).
 constexpr int kPWarps = 4, kVWarps = 4;
-// The sender slices of the block kPrefetch ahead are prefetched into L2 (by the warp that will
-// load each chunk), so that the ring's loads find them there: the ring holds only ~1.5 blocks,
-// too few bytes in flight to cover the HBM latency on its own.
-constexpr int kPrefetch = 3;
 constexpr int kND = 8;           // mixing-result TMEM slots (chunks)
 constexpr int kNG = kND / 2;     // ... committed and released in pairs of chunks (one commit costs
                                  // ~90 ns of issue time on this B200, an MMA ~25 ns)
@@ -217,23 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
       const uint64_t pol = tc::policy_evict_first();   // each stored tile is read once
       if (pw == 0)
         for (int i = 0; i < 8; ++i) tc::prefetch_tmap(&p.p_maps[i]);
-      // L2 prefetch of this warp's chunks of block tb
-      auto prefetch_block = [&](int tb) {
-        const unsigned long long mp = p.headmask[u0 + tb];
-        const int kp = __popcll(mp);
-        const int yp = (int)(p.val_off[u0 + tb] * 64);
-        const CUtensorMap* mapp = &p.p_maps[((kp + 7) >> 3) - 1];
-        for (int c = 0; c < nch; ++c) {
-          if ((tb * nch + c) % kPWarps != pw) continue;
-          tc::tma_prefetch_2d(mapp, 0, yp + (2 * (c0 + c)) * kp);
-          tc::tma_prefetch_2d(mapp, 0, yp + (2 * (c0 + c) + 1) * kp);
-        }
-      };
-      for (int tb = 1; tb <= kPrefetch && tb < T; ++tb) prefetch_block(tb);
       unsigned long long m_next = T > 0 ? p.headmask[u0] : 0ull;
       int64_t off_next = T > 0 ? p.val_off[u0] : 0;
       for (int t = 0; t < T; ++t) {
-        if (t + kPrefetch + 1 < T) prefetch_block(t + kPrefetch + 1);
         const unsigned long long m = m_next;
         const int64_t off = off_next;
         if (t + 1 < T) {

@@ -119,14 +119,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Prefetch of a 2-D tile into L2 (no shared memory, no completion): the tile a later
-// tma_load_2d of the same map and coordinates reads then comes from L2.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map),
-               "r"(x), "r"(y)
-               : "memory");
-}
-
 // Brings a tensor map (kernel parameter) into the TMA unit's descriptor cache.
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");

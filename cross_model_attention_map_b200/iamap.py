@@ -85,6 +85,12 @@ _SIGS = {
     "iamap_compress_with_output": (_I, [_P, _P, _P, _P, _I, _I64, _I, _I, _I, _F, _I, _F,
                                         _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64,
                                         _P, _SZ, _P]),
+    "iamap_compress_extract_with_output": (_I, [_P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _F,
+                                                _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P,
+                                                _SZ, _P]),
+    "iamap_sender_rows_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "iamap_sender_rows": (_I, [_P, _P, _I64, _P, _I, _I, _P, _P, _I, _I, _I, _P, _I, _P, _SZ,
+                               _P]),
     "iamap_chunk_plan": (_I, [_P, _P, _P, _I, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
                               ctypes.POINTER(ctypes.c_int32)]),
     "iamap_compress_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I64, _I64, _I, _I, _I,
@@ -252,6 +258,33 @@ def iamap_prefill_steps_host(q_host, k_host, v_host, W_host, out_host, cu_seqlen
         _ptr(counts), _ptr(vals), vals_capacity_tiles, _ptr(io), io.numel() * io.element_size(),
         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
     del keep, arrs
+
+
+def iamap_compress_extract_with_output(q, k, cu_seqlens, cu_seqlens_host, num_seqs, n, H_s, d,
+                                       B, bias_window, bias_value, v_s, d_vs, o_s, lse, row_ptr,
+                                       col_idx, headmask, val_off, counts, vals,
+                                       vals_capacity_tiles, ws, stream=None):
+    cp, keep = _host_i32(cu_seqlens_host)
+    _check("iamap_compress_extract_with_output", _lib.iamap_compress_extract_with_output(
+        _ptr(q), _ptr(k), _ptr(cu_seqlens), cp, num_seqs, n, H_s, d, B, bias_window, bias_value,
+        _ptr(v_s), d_vs, _ptr(o_s), _ptr(lse), _ptr(row_ptr), _ptr(col_idx), _ptr(headmask),
+        _ptr(val_off), _ptr(counts), _ptr(vals), vals_capacity_tiles, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def iamap_sender_rows_workspace_bytes(batch, H_s, ctx_stride) -> int:
+    return _lib.iamap_sender_rows_workspace_bytes(batch, H_s, ctx_stride)
+
+
+def iamap_sender_rows(q, k_pages, num_pages, page_table, max_pages, page_size, ctx_lens,
+                      ctx_lens_host, batch, H_s, d, p_rows, ctx_stride, ws, stream=None):
+    cp, keep = _host_i32(ctx_lens_host)
+    _check("iamap_sender_rows", _lib.iamap_sender_rows(
+        _ptr(q), _ptr(k_pages), num_pages, _ptr(page_table), max_pages, page_size,
+        _ptr(ctx_lens), cp, batch, H_s, d, _ptr(p_rows), ctx_stride, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
 
 
 def iamap_chunk_plan(cu_q_host, cu_k_host, starts_host, num_seqs, B):

@@ -15,7 +15,8 @@
  *                combination of sender heads is in its layer/head-mapping paragraph.)
  *   mapped_av_paged  the decode form: one query row per sequence, sender rows given, V in a paged
  *                cache. ("IAM: Efficient Inference through Attention Mapping between
- *                Different-scale LLMs" notes, Method section 4, decode bullet.)
+ *                Different-scale LLMs" notes, Method section 4, decode bullet.) The sender rows
+ *                themselves: iamap_sender_rows (the small model's softmax row, paged keys).
  *   head_match   IAM's calibration: cosine similarity of flattened causal attention maps of every
  *                large-model head with every small-model head, then the most similar small head
  *                per large head. (IAM notes, Method sections 1 and 4.) Variants: Pearson and
@@ -218,6 +219,22 @@ int iamap_compress_with_output(const void* q, const void* k, const int32_t* cu_s
                                void* stream);
 
 /*
+ * Compress stage 2 with the sender's own attention output: as iamap_compress_extract (on the
+ * outputs of iamap_compress_stats), and in the same pass the sender output o_s of
+ * iamap_compress_with_output. Lets a caller read the tile count after stage 1 and allocate the
+ * value buffer exactly. Sequences may hold at most 256 blocks of 64.
+ */
+int iamap_compress_extract_with_output(const void* q, const void* k, const int32_t* cu_seqlens,
+                                       const int32_t* cu_seqlens_host, int num_seqs, int64_t n,
+                                       int H_s, int d, int B, int bias_window, float bias_value,
+                                       const void* v_s, int d_vs, float* o_s, const float* lse,
+                                       const int32_t* row_ptr, const int32_t* col_idx,
+                                       const uint64_t* headmask, const int64_t* val_off,
+                                       const int64_t* counts, void* vals,
+                                       int64_t vals_capacity_tiles, void* ws, size_t ws_bytes,
+                                       void* stream);
+
+/*
  * Chunked prefill ("PKU MapFlow" news page, the paragraph on the vLLM integration: the fused
  * kernel works with chunked prefill). Sequence s of a batch has keys [0, e_s), e_s =
  * cu_k[s+1] - cu_k[s], and a chunk of query rows [starts[s], e_s); starts[s] is a multiple of
@@ -298,6 +315,25 @@ int iamap_prefill_steps_host(int steps, const void* const* q_host, const void* c
                              int64_t* val_off, int64_t* counts, void* vals,
                              int64_t vals_capacity_tiles, void* io, size_t io_bytes, void* ws,
                              size_t ws_bytes, void* stream);
+
+/*
+ * The small model's attention row of a decode step, the row a mapped layer reuses (IAM notes,
+ * Method section 4, decode bullet): p[b, h, j] = softmax over j < ctx_lens[b] of
+ * q[b, h] . k[b, j, h] / sqrt(d), keys in a paged cache.
+ *   q        bf16 [batch, H_s, d]                   (d a multiple of 8, at most 128)
+ *   k_pages  bf16 [num_pages, page_size, H_s, d]    16-byte aligned; key j of sequence b is
+ *            row j % page_size of page page_table[b, j / page_size]
+ *   p_rows   fp32 [batch, H_s, ctx_stride]          written in full (zeros at j >= ctx_lens[b])
+ *   ws       iamap_sender_rows_workspace_bytes bytes (per-chunk partial sums)
+ * A page index outside [0, num_pages) makes that key's probability 0 and sets
+ * IAMAP_DEV_BAD_INDEX. The result feeds iamap_mapped_av_paged as its p_rows.
+ */
+size_t iamap_sender_rows_workspace_bytes(int batch, int H_s, int ctx_stride);
+int iamap_sender_rows(const void* q, const void* k_pages, int64_t num_pages,
+                      const int32_t* page_table, int max_pages, int page_size,
+                      const int32_t* ctx_lens, const int32_t* ctx_lens_host, int batch, int H_s,
+                      int d, float* p_rows, int ctx_stride, void* ws, size_t ws_bytes,
+                      void* stream);
 
 /*
  * Decode step on a mapped layer: one query row per sequence b.

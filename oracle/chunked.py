@@ -177,6 +177,8 @@ def sender_output(wl, v_s: np.ndarray) -> np.ndarray:
     O = np.zeros((wl.n, wl.H_s, v_s.shape[2]))
     for s in range(len(wl.seqlens)):
         a, b = int(wl.cu_seqlens[s]), int(wl.cu_seqlens[s + 1])
+        if b == a:
+            continue   # an empty sequence has no rows
         for h in range(wl.H_s):
             O[a:b, h] = _sender_rows(head_rows(wl.q, a, b, h), head_rows(wl.k, a, b, h),
                                      bf16_bits_to_f64(v_s[a:b, h]), 0, wl.bias_window,
@@ -193,6 +195,8 @@ def sender_output_chunk(cw, v_s_keys: np.ndarray) -> np.ndarray:
         ka, e = int(cw.cu_k[s]), lay.ends[s]
         qa, qb = int(cw.cu_q[s]), int(cw.cu_q[s + 1])
         c0 = lay.I0[s] * cw.B
+        if qb == qa:
+            continue   # a chunk with no query rows
         for h in range(cw.H_s):
             O[qa:qb, h] = _sender_rows(head_rows(cw.q, qa, qb, h), head_rows(cw.k, ka, ka + e, h),
                                        bf16_bits_to_f64(v_s_keys[ka:ka + e, h]), c0,

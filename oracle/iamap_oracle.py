@@ -60,6 +60,7 @@ __all__ = [
     "block_masses", "select_blocks", "RowBlockStats", "rowblock_stats", "CompressResult",
     "compress", "union_bsr", "masked_tile", "mapped_av_rows", "mapped_av", "mapped_av_paged",
     "attention_map", "head_match", "mapping_consistency", "receiver_values",
+    "sender_decode_rows",
 ]
 
 
@@ -345,6 +346,27 @@ def mapped_av(wl, kept: np.ndarray) -> np.ndarray:
             rows = mapped_av_rows(wl, s, I, lambda h: kept[h, c0:c0 + I + 1])
             O[a + I * wl.B:a + I * wl.B + rows.shape[0]] = rows
     return O
+
+
+def sender_decode_rows(dw) -> np.ndarray:
+    """The small model's attention row of a decode step [IAM-4] (the row a mapped layer reuses)
+    and the textbook softmax of scaled dot products [GLIDE II-B]: p[b, h, j] = softmax over
+    j < ctx_len[b] of q_s[b, h] . k_s[b, j, h] / sqrt(d_s), the keys gathered through the page
+    table. Returns float64 [batch, H_s, max_ctx] with zeros at j >= ctx_len[b]."""
+    d = dw.q_s.shape[2]
+    max_ctx = int(np.max(dw.ctx_lens))
+    P = np.zeros((dw.batch, dw.H_s, max_ctx))
+    ps = dw.page_size
+    for b in range(dw.batch):
+        c = int(dw.ctx_lens[b])
+        if c == 0:
+            continue
+        pages = dw.page_table[b, (np.arange(c) // ps)]
+        K = bf16_bits_to_f64(dw.k_pages_s[pages, np.arange(c) % ps])      # [c, H_s, d]
+        q = bf16_bits_to_f64(dw.q_s[b])                                      # [H_s, d]
+        s = np.einsum("hd,jhd->hj", q, K) / math.sqrt(d)
+        P[b, :, :c], _ = softmax_rows(s)
+    return P
 
 
 def mapped_av_paged(dw) -> np.ndarray:

@@ -207,16 +207,22 @@ class DecodeWorkload:
     assign: np.ndarray      # int32 [H_r]: the sender head of each receiver head
     v_pages: np.ndarray     # uint16 bf16 [num_pages, page_size, H_r, d_v]
     page_table: np.ndarray  # int32 [batch, max_pages]
+    q_s: np.ndarray = None        # uint16 bf16 [batch, H_s, d_s]: the small model's query
+    k_pages_s: np.ndarray = None  # uint16 bf16 [num_pages, page_size, H_s, d_s]: its keys, on
+                                  # the same pages as the large model's values
 
 
 def make_decode(batch=4, ctx=8704, H_s=14, H_r=64, d_v=128, page_size=16, sink_weight=64.0,
-                ctx_lens=None, seed=0, H_kv=None) -> DecodeWorkload:
-    """Draw order: sender rows, one-hot assignment, V pages, page-table permutation.
+                ctx_lens=None, seed=0, H_kv=None, d_s=64) -> DecodeWorkload:
+    """Draw order: sender rows, one-hot assignment, V pages, page-table permutation, the small
+    model's query, its key pages.
 
-    The sender's attention rows are drawn from a Dirichlet distribution (normalised Gamma draws)
-    with a heavier concentration at position 0, a stand-in for a causal softmax row with a sink.
-    Unused tail positions (ctx_len < max) are zero. ``H_kv`` (dividing H_r) gives the page
-    pool that many value heads.
+    ``p_rows`` are drawn from a Dirichlet distribution (normalised Gamma draws) with a heavier
+    concentration at position 0 (unused tail positions, ctx_len < max, are zero): an extra case
+    of given rows. The configuration's rows are the small model's own softmax rows over its keys:
+    ``q_s`` and ``k_pages_s`` (N(0, 1), head dim d_s, keys on the same pages as the values) are
+    the inputs from which they are computed. ``H_kv`` (dividing H_r) gives the page pool that many
+    value heads.
     """
     if ctx_lens is None:
         ctx_lens = [ctx] * batch
@@ -239,9 +245,12 @@ def make_decode(batch=4, ctx=8704, H_s=14, H_r=64, d_v=128, page_size=16, sink_w
                             dtype=np.float32)
     perm = rng.permutation(num_pages).astype(np.int32)
     page_table = perm.reshape(batch, max_pages)
+    q_s = rng.standard_normal((batch, H_s, d_s), dtype=np.float32)
+    k_s = rng.standard_normal((num_pages, page_size, H_s, d_s), dtype=np.float32)
     return DecodeWorkload(batch=batch, ctx_lens=ctx_lens, H_s=H_s, H_r=H_r, d_v=d_v,
                           page_size=page_size, p_rows=p_rows, W=W, assign=assign,
-                          v_pages=bf16_bits(v), page_table=page_table)
+                          v_pages=bf16_bits(v), page_table=page_table, q_s=bf16_bits(q_s),
+                          k_pages_s=bf16_bits(k_s))
 
 
 def decode_config(seed: int = 0) -> DecodeWorkload:

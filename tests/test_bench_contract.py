@@ -3,6 +3,8 @@ host) prints one JSON line with the contract's keys; under torchrun only rank 0 
 than 3 warm-up steps are refused."""
 
 import json
+
+import numpy as np
 import os
 import subprocess
 import sys
@@ -66,3 +68,38 @@ def test_oracle_timing_helpers_on_small_workloads():
     dw = make_decode(batch=2, ctx=100, H_s=3, H_r=4, d_v=16, seed=1)
     rows, dt = bench.oracle_decode_step(dw)
     assert abs(rows * dt - 2) < 1e-9
+
+
+def test_reference_arm_prefill_times_what_it_reports():
+    """The prefill reference arm times one row block of a fixed, stated sample per step, and its
+    ms_per_step is that measured time (so steps x ms_per_step fits inside the run)."""
+    import time
+    t0 = time.time()
+    r = _run(["--impl", "reference", "--config", "tiny", "--steps", "3", "--warmup", "3"])
+    wall = time.time() - t0
+    assert r.returncode == 0, r.stderr
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["steps"] * d["ms_per_step"] / 1e3 <= wall
+    assert "fixed sample" in d["cpu_baseline"]["sample"]
+    assert d["ms_per_workload_extrapolated"] > 0
+
+
+def test_kept_set_check_counts_a_planted_mismatch():
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle as O
+    from synth import make_prefill
+    wl = make_prefill([300, 200], H_s=3, d=32, H_r=2, d_v=8, B=64, tau=0.9, seed=79)
+    blocks = bench.systematic_rowblocks(wl, 3)
+    assert len(blocks) == 3 and len(set(blocks)) == 3
+    _, rows, _, stats, text = bench.oracle_sample_prefill(wl, blocks)
+    kept = O.compress(wl).kept
+    chk = bench.kept_set_check(wl, kept, stats)
+    assert chk["mismatches_outside_near"] == 0 and chk["flips"] == 0
+    assert chk["blocks"] == 3 * sum(I + 1 for _, I in blocks)
+    s, I = blocks[1]
+    lay = O.causal_layout(wl.seqlens, wl.B)
+    J = int(np.flatnonzero(stats[1][2][0].kept)[0])
+    bad = kept.copy()
+    bad[0, lay.cb(s, I, J)] = False
+    assert bench.kept_set_check(wl, bad, stats)["mismatches_outside_near"] == 1

@@ -125,3 +125,19 @@ def test_chunk_start_must_be_a_block_multiple():
     wl = make_prefill([64], H_s=1, d=16, H_r=1, d_v=8, B=16, seed=10)
     with pytest.raises(ValueError):
         CH.compress_chunk(chunk_of(wl, [8]))
+
+
+def test_sender_output_of_empty_sequences_and_chunks():
+    """Sequences and chunks without rows contribute no output rows (and do not disturb the
+    others): the other sequences' rows equal those of the batch without the empty ones."""
+    wl = make_prefill([40, 0, 20], H_s=2, d=16, H_r=2, d_v=8, B=16, seed=6)
+    vs = make_sender_values(wl, d_vs=8)
+    out = CH.sender_output(wl, vs)
+    assert out.shape == (60, 2, 8)
+    from synth import select_sequences
+    sub = select_sequences(wl, [0, 2])
+    np.testing.assert_array_equal(out, CH.sender_output(sub, np.concatenate([vs[:40], vs[40:]])))
+    cw = chunk_of(wl, [16, 0, 16], [40, 0, 20])
+    oc = CH.sender_output_chunk(cw, np.concatenate([vs[:40], vs[40:60]]))
+    np.testing.assert_allclose(oc[:24], out[16:40], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(oc[24:], out[56:60], rtol=1e-12, atol=1e-14)

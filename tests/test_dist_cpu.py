@@ -146,3 +146,81 @@ def test_prefill_split_by_sequence_equals_whole_batch():
                 c = int(sub.cu_seqlens[i])
                 np.testing.assert_array_equal(o[c:c + b - a], whole[a:b])
                 np.testing.assert_array_equal(r.lse[:, c:c + b - a], res.lse[:, a:b])
+
+
+def _bench_sequence_split(rank, world, port, out):
+    """The host side of `bench.py --split seq`: each rank takes its sequences of one packed batch
+    (a rank without any follows the same barriers and max reductions with zero time), and the
+    step time is the max over ranks."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth import make_prefill
+    _init(rank, world, port)
+    try:
+        wl = make_prefill([300, 64, 700, 5], H_s=2, d=16, H_r=2, d_v=8, B=64, tau=0.9, seed=77)
+        sub, mine = bench.split_by_sequence(wl, world, rank)
+        rows = {s: sub.q[int(sub.cu_seqlens[i]):int(sub.cu_seqlens[i + 1])].tobytes()
+                for i, s in enumerate(mine)}
+        bench.barrier(world)
+        bench.barrier(world)
+        ms = bench.max_over_ranks(10.0 * (rank + 1), world)
+        bench.barrier(world)
+        e2e = bench.max_over_ranks(1.0 + rank, world)
+        out[rank] = (mine, sub.n, {s: r for s, r in rows.items()}, ms, e2e)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_sequence_split_world2():
+    import sys
+    sys.path.insert(0, ROOT)
+    from synth import make_prefill
+    out = _run(_bench_sequence_split)
+    wl = make_prefill([300, 64, 700, 5], H_s=2, d=16, H_r=2, d_v=8, B=64, tau=0.9, seed=77)
+    mine0, n0, rows0, ms0, e0 = out[0]
+    mine1, n1, rows1, ms1, e1 = out[1]
+    # every sequence on exactly one rank; the longest (700 tokens, 66 causal blocks) alone on
+    # rank 0, the rest (15 + 1 + 1 blocks) on rank 1
+    assert sorted(mine0 + mine1) == [0, 1, 2, 3]
+    assert mine0 == [2] and mine1 == [0, 1, 3]
+    assert n0 + n1 == wl.n
+    # each rank's rows are the packed batch's rows of its sequences (slices, bit for bit)
+    for rows in (rows0, rows1):
+        for s, r in rows.items():
+            a, b = int(wl.cu_seqlens[s]), int(wl.cu_seqlens[s + 1])
+            assert r == wl.q[a:b].tobytes()
+    assert ms0 == ms1 == 20.0 and e0 == e1 == 2.0
+
+
+def _bench_idle_rank(rank, world, port, out):
+    """A rank with no sequence (4 ranks, 2 sequences) takes the working ranks' collectives."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import argparse
+    import bench
+    from synth import make_prefill
+    _init(rank, world, port)
+    try:
+        wl = make_prefill([200, 70], H_s=2, d=16, H_r=2, d_v=8, B=64, tau=0.9, seed=78)
+        sub, mine = bench.split_by_sequence(wl, world, rank)
+        if not mine:
+            r = bench.idle_rank(argparse.Namespace(), world, wl.n)
+            out[rank] = ("idle", r["ms"], r["e2e_ms"])
+        else:
+            bench.barrier(world)
+            bench.barrier(world)
+            ms = bench.max_over_ranks(3.0 + rank, world)
+            bench.barrier(world)
+            e2e = bench.max_over_ranks(4.0 + rank, world)
+            out[rank] = (mine, ms, e2e)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_sequence_split_idle_ranks():
+    out = _run(_bench_idle_rank, world=4)
+    assert out[0][0] == [0] and out[1][0] == [1]
+    assert out[2][0] == "idle" and out[3][0] == "idle"
+    for r in range(4):
+        assert out[r][-2] == 4.0 and out[r][-1] == 5.0

@@ -221,3 +221,29 @@ def test_varlen40k_chunks_sampled(C):
         ref = O.mapped_av_rows(wl, s, I, lambda h: kept[h, b0:b0 + I + 1], lambda h: st[h])
         r0 = int(cw.cu_q[s]) + I * wl.B - starts[s]
         check_output(out[r0:r0 + ref.shape[0]], ref, "chunk rows of block (%d, %d)" % (s, I))
+
+
+def test_two_phase_extract_with_output(C):
+    """Stats, read the tile count, allocate exactly, then extract with the sender output: the same
+    tiles and the same sender output as the one-call iamap_compress_with_output."""
+    from cross_model_attention_map_b200.runner import PrefillLayer
+    wl = make_prefill([500, 180], H_s=6, d=128, H_r=4, d_v=64, B=64, tau=0.9, seed=65)
+    v_s = make_sender_values(wl)
+    one, o_one = _whole(wl, v_s)
+    q, k, v, W = upload_prefill(wl)
+    two = PrefillLayer(wl.seqlens, 6, 128, 4, 64, 0.9, capacity_tiles=1)
+    b = two.bufs
+    C.iamap_compress_stats(q, k, two.cu, two.cu_host, two.num_seqs, two.n, 6, 128, 64, 0.9, 0, 0.0,
+                           b["lse"], b["mass"], b["headmask_dense"], b["row_ptr"], b["col_idx"],
+                           b["headmask"], b["val_off"], b["counts"], two.ws)
+    nnz, tiles = two.counts()
+    vals = torch.empty(tiles, 64, 64, dtype=torch.bfloat16, device="cuda")
+    o_s = torch.empty(wl.n, 6, 128, dtype=torch.float32, device="cuda")
+    C.iamap_compress_extract_with_output(q, k, two.cu, two.cu_host, two.num_seqs, two.n, 6, 128,
+                                         64, 0, 0.0, bf16(v_s), 128, o_s, b["lse"], b["row_ptr"],
+                                         b["col_idx"], b["headmask"], b["val_off"], b["counts"],
+                                         vals, tiles, two.ws)
+    torch.cuda.synchronize()
+    assert C.iamap_device_status() == 0
+    assert torch.equal(vals, one.vals[:tiles])
+    assert torch.equal(o_s, o_one)

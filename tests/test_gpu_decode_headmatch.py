@@ -29,13 +29,70 @@ def _run_decode(dw):
     return out.cpu().numpy()
 
 
+def _gpu_sender_rows(C, dw):
+    """The small model's decode rows on the GPU (iamap_sender_rows), as a device tensor."""
+    max_ctx = int(dw.ctx_lens.max())
+    rows = torch.empty(dw.batch, dw.H_s, max_ctx, dtype=torch.float32, device="cuda")
+    ws = C.alloc_workspace(C.iamap_sender_rows_workspace_bytes(dw.batch, dw.H_s, max_ctx))
+    C.iamap_sender_rows(bf16(dw.q_s), bf16(dw.k_pages_s), dw.k_pages_s.shape[0],
+                        torch.from_numpy(dw.page_table).cuda(), dw.page_table.shape[1],
+                        dw.page_size, torch.from_numpy(dw.ctx_lens).cuda(), dw.ctx_lens,
+                        dw.batch, dw.H_s, dw.q_s.shape[2], rows, max_ctx, ws)
+    torch.cuda.synchronize()
+    return rows
+
+
+def test_sender_rows_parity(C):
+    """The small model's decode rows (softmax of q.k / 8 over 8704 paged keys, 14 heads) against
+    the oracle: relative error of every row within the output tolerance, rows summing to 1."""
+    dw = decode_config()
+    rows = _gpu_sender_rows(C, dw).cpu().numpy()
+    assert C.iamap_device_status() == 0
+    ref = O.sender_decode_rows(dw)
+    for b in range(dw.batch):
+        check_output(rows[b], ref[b], "sender rows of sequence %d" % b)
+    np.testing.assert_allclose(rows.sum(axis=2), 1.0, rtol=0, atol=1e-4)
+
+
+def test_sender_rows_ragged_and_bad_page(C):
+    dw = make_decode(batch=4, ctx=600, H_s=3, H_r=4, d_v=64, page_size=16,
+                     ctx_lens=[600, 0, 17, 513], seed=34, d_s=128)
+    rows = _gpu_sender_rows(C, dw).cpu().numpy()
+    assert C.iamap_device_status() == 0
+    ref = O.sender_decode_rows(dw)
+    for b in (0, 2, 3):
+        check_output(rows[b], ref[b], "sender rows of sequence %d" % b)
+    assert np.all(rows[1] == 0) and np.all(rows[2, :, 17:] == 0)
+    dw.page_table[3, 5] = dw.k_pages_s.shape[0] + 7          # a page outside the pool
+    rows = _gpu_sender_rows(C, dw).cpu().numpy()
+    assert C.iamap_device_status() & C.IAMAP_DEV_BAD_INDEX
+    assert np.all(rows[3, :, 80:96] == 0)
+
+
 def test_decode_config_parity(C):
     """Batch 4, context 8704, 14 sender heads, 64 receiver heads d_v=128, one-hot W, 16-token
-    pages under a random page table."""
+    pages under a random page table; the sender rows are the small model's own softmax rows,
+    computed on the GPU (iamap_sender_rows) and compared with the oracle's output on the
+    oracle's rows."""
+    dw = decode_config()
+    gpu_rows = _gpu_sender_rows(C, dw)
+    from cross_model_attention_map_b200.runner import DecodeStep
+    st = DecodeStep(dw.batch, dw.H_s, dw.H_r, dw.d_v, dw.ctx_lens, gpu_rows.shape[2],
+                    dw.page_table.shape[1], dw.page_size, dw.v_pages.shape[0])
+    out = st.run(gpu_rows, torch.from_numpy(dw.W).cuda(), bf16(dw.v_pages),
+                 torch.from_numpy(dw.page_table).cuda())
+    torch.cuda.synchronize()
+    assert C.iamap_device_status() == 0
+    dw.p_rows = O.sender_decode_rows(dw)
+    check_output(out.cpu().numpy(), O.mapped_av_paged(dw), "paged decode")
+
+
+def test_decode_dirichlet_rows(C):
+    """The same step on given rows (Dirichlet draws with a sink at position 0)."""
     dw = decode_config()
     out = _run_decode(dw)
     assert C.iamap_device_status() == 0
-    check_output(out, O.mapped_av_paged(dw), "paged decode")
+    check_output(out, O.mapped_av_paged(dw), "paged decode, given rows")
 
 
 def test_decode_ragged_general_W(C):

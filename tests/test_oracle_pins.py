@@ -525,3 +525,23 @@ def test_grouped_values_equal_repeated_heads():
     np.testing.assert_array_equal(O.mapped_av_paged(dw), O.mapped_av_paged(drep))
     with pytest.raises(ValueError):
         O.receiver_values(np.zeros((3, 4, 2)), 6)
+
+
+def test_sender_decode_rows_equal_torch_softmax():
+    """The small model's decode rows: torch's float64 softmax of the scaled dot products of the
+    query with the keys, gathered here by plain indexing of the page pool (no page-table walk),
+    rows of different context lengths, zeros past each length."""
+    dw = make_decode(batch=3, ctx=70, H_s=2, H_r=4, d_v=8, page_size=16, ctx_lens=[70, 5, 33],
+                     seed=13, d_s=16)
+    P = O.sender_decode_rows(dw)
+    assert P.shape == (3, 2, 70)
+    q = torch.from_numpy(bf16_bits_to_f64(dw.q_s))
+    K = torch.from_numpy(bf16_bits_to_f64(dw.k_pages_s))
+    for b in range(3):
+        c = int(dw.ctx_lens[b])
+        keys = torch.stack([K[int(dw.page_table[b, j // 16]), j % 16] for j in range(c)])  # [c, H, d]
+        logits = torch.einsum("hd,jhd->hj", q[b], keys) / 4.0
+        np.testing.assert_allclose(P[b, :, :c], torch.softmax(logits, dim=1).numpy(),
+                                   rtol=1e-12, atol=1e-15)
+        assert (P[b, :, c:] == 0).all()
+        np.testing.assert_allclose(P[b, :, :c].sum(axis=1), 1.0, rtol=0, atol=1e-12)
