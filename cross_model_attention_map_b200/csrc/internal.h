@@ -89,6 +89,9 @@ struct MappedAvArgs {
   // Chunked prefill: v holds n_k tokens packed by cu_seqlens (the keys of every sequence), out
   // the n query rows of the chunks (SeqTables::qoff); 0 = v and out alike.
   int64_t n_k = 0;
+  // Several mapped layers in one launch: sequence s uses the mixing matrix W + (s / seqs_per_w)
+  // * H_r * H_s (0 = one W for every sequence).
+  int seqs_per_w = 0;
 };
 int mapped_av_impl(const MappedAvArgs& a, cudaStream_t stream);
 // Tensor-core, cluster-cooperative form (mapped_av_tc.cu); used when supported.

@@ -38,6 +38,7 @@ struct AvParams {
   const __nv_bfloat16* vals;
   int64_t capacity;
   const float* W;
+  int seqs_per_w;   // sequences per mixing matrix (several layers per launch; 0 = one W)
   const __nv_bfloat16* v;
   float* out;
   unsigned int* status;
@@ -74,10 +75,11 @@ __global__ void __launch_bounds__(kAvThreads, 1) mapped_av_kernel(AvParams p) {
   const int G = min(kAvGroup, p.H_r - r0);
   const int64_t vrs = (int64_t)p.H_kv * DV;  // V row stride (elements)
   const int kv_grp = p.H_r / p.H_kv;
+  const float* Wl = p.W + (p.seqs_per_w ? (int64_t)(s / p.seqs_per_w) * p.H_r * p.H_s : 0);
 
   for (int e = tid; e < kAvGroup * 64; e += kAvThreads) {
     const int r = e / 64, hs = e % 64;
-    sW[e] = (r < G && hs < p.H_s) ? p.W[(int64_t)(r0 + r) * p.H_s + hs] : 0.f;
+    sW[e] = (r < G && hs < p.H_s) ? Wl[(int64_t)(r0 + r) * p.H_s + hs] : 0.f;
   }
 
   // PV role of this warp: 16 rows, one receiver head of the group.
@@ -255,6 +257,7 @@ int mapped_av_impl(const MappedAvArgs& a, cudaStream_t stream) {
   p.vals = static_cast<const __nv_bfloat16*>(a.vals);
   p.capacity = a.capacity;
   p.W = a.W;
+  p.seqs_per_w = a.seqs_per_w;
   p.v = static_cast<const __nv_bfloat16*>(a.v);
   p.out = a.out;
   p.status = a.status;

@@ -139,6 +139,7 @@ struct __align__(64) Params {
   unsigned int* status;
   int H_s, H_r, d_v, C, NR, KH, RB, NP;
   int grp;                 // receiver heads per value head (grouped values; 1 = one each)
+  int seqs_per_w;          // sequences per mixing matrix (several layers per launch; 0 = one W)
   uint32_t off_p, off_w, off_scr, off_recv, off_v, off_wf, off_bar;
 };
 
@@ -191,9 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
     const int nz = (int)((NP * p_stage + 1024u) / 16);
     for (int i = tid; i < nz; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
     float* wf = reinterpret_cast<float*>(smem + p.off_wf);   // W transposed: [H_s][H_r]
+    const float* Wl = p.W + (p.seqs_per_w ? (int64_t)(s / p.seqs_per_w) * p.H_r * p.H_s : 0);
     for (int i = tid; i < p.H_r * p.H_s; i += kThreads) {
       const int r = i / p.H_s, h = i - r * p.H_s;
-      wf[h * p.H_r + r] = p.W[i];
+      wf[h * p.H_r + r] = Wl[i];
     }
     tc::fence_proxy_async_smem();
   }
@@ -561,6 +563,7 @@ int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream) {
   p.headmask = reinterpret_cast<const unsigned long long*>(a.headmask);
   p.val_off = a.val_off;
   p.W = a.W;
+  p.seqs_per_w = a.seqs_per_w;
   p.out = a.out;
   p.status = a.status;
 

@@ -91,6 +91,13 @@ _SIGS = {
     "iamap_sender_rows_workspace_bytes": (_SZ, [_I, _I, _I]),
     "iamap_sender_rows": (_I, [_P, _P, _I64, _P, _I, _I, _P, _P, _I, _I, _I, _P, _I, _P, _SZ,
                                _P]),
+    "iamap_layers_plan": (_I, [_P, _I, _I, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
+                               ctypes.POINTER(ctypes.c_int32)]),
+    "iamap_layers_workspace_bytes": (_SZ, [_I, _I, _I64]),
+    "iamap_compress_layers": (_I, [_P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _F, _I, _F, _P, _P,
+                                   _P, _P, _P, _P, _P, _P, _P, _I64, _P, _SZ, _P]),
+    "iamap_mapped_av_layers": (_I, [_P, _P, _I, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _I64, _P,
+                                    _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "iamap_chunk_plan": (_I, [_P, _P, _P, _I, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
                               ctypes.POINTER(ctypes.c_int32)]),
     "iamap_compress_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I64, _I64, _I, _I, _I,
@@ -284,6 +291,44 @@ def iamap_sender_rows(q, k_pages, num_pages, page_table, max_pages, page_size, c
         _ptr(q), _ptr(k_pages), num_pages, _ptr(page_table), max_pages, page_size,
         _ptr(ctx_lens), cp, batch, H_s, d, _ptr(p_rows), ctx_stride, _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def iamap_layers_plan(cu_seqlens_host, num_seqs, num_layers, B):
+    cp, keep = _host_i32(cu_seqlens_host)
+    nrb, ncb, mx = _I64(0), _I64(0), ctypes.c_int32(0)
+    _check("iamap_layers_plan", _lib.iamap_layers_plan(cp, num_seqs, num_layers, B,
+                                                       ctypes.byref(nrb), ctypes.byref(ncb),
+                                                       ctypes.byref(mx)))
+    del keep
+    return nrb.value, ncb.value, mx.value
+
+
+def iamap_layers_workspace_bytes(num_seqs, num_layers, num_rowblocks) -> int:
+    return _lib.iamap_layers_workspace_bytes(num_seqs, num_layers, num_rowblocks)
+
+
+def iamap_compress_layers(q, k, cu_seqlens, cu_seqlens_host, num_seqs, n, num_layers, H_s, d, B,
+                          tau, bias_window, bias_value, lse, mass, headmask_dense, row_ptr,
+                          col_idx, headmask, val_off, counts, vals, vals_capacity_tiles, ws,
+                          stream=None):
+    cp, keep = _host_i32(cu_seqlens_host)
+    _check("iamap_compress_layers", _lib.iamap_compress_layers(
+        _ptr(q), _ptr(k), _ptr(cu_seqlens), cp, num_seqs, n, num_layers, H_s, d, B, tau,
+        bias_window, bias_value, _ptr(lse), _ptr(mass), _ptr(headmask_dense), _ptr(row_ptr),
+        _ptr(col_idx), _ptr(headmask), _ptr(val_off), _ptr(counts), _ptr(vals),
+        vals_capacity_tiles, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def iamap_mapped_av_layers(cu_seqlens, cu_seqlens_host, num_seqs, n, num_layers, B, H_s, row_ptr,
+                           col_idx, headmask, val_off, vals, vals_capacity_tiles, W, H_r, H_kv, v,
+                           d_v, out, ws, stream=None):
+    cp, keep = _host_i32(cu_seqlens_host)
+    _check("iamap_mapped_av_layers", _lib.iamap_mapped_av_layers(
+        _ptr(cu_seqlens), cp, num_seqs, n, num_layers, B, H_s, _ptr(row_ptr), _ptr(col_idx),
+        _ptr(headmask), _ptr(val_off), _ptr(vals), vals_capacity_tiles, _ptr(W), H_r, H_kv,
+        _ptr(v), d_v, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
     del keep
 
 

@@ -24,6 +24,7 @@
  *                (section 3).
  *   *_gqa        mapped_av / mapped_av_paged with grouped receiver values: H_kv value heads,
  *                receiver head r reads value head r / (H_r / H_kv).
+ *   *_layers     several mapped layer pairs per launch (layer-major stacked tensors).
  *   prefill_steps_host  end-to-end steps on host-resident inputs, the copies overlapping the
  *                kernels of neighbouring steps.
  *   compress_with_output, *_chunk  the sender's own attention output fused into compress, and
@@ -233,6 +234,39 @@ int iamap_compress_extract_with_output(const void* q, const void* k, const int32
                                        const int64_t* counts, void* vals,
                                        int64_t vals_capacity_tiles, void* ws, size_t ws_bytes,
                                        void* stream);
+
+/*
+ * Several mapped layer pairs in one launch per stage ("PKU MapFlow" news page, the layer/head-
+ * mapping paragraph: receiver layers paired with sender layers). num_layers = L pairs over the
+ * same packed sequences (cu_seqlens, n tokens, S = num_seqs): the layers' tensors are stacked
+ * layer-major,
+ *   q, k  bf16 [L, n, H_s, d]       v  bf16 [L, n, H_kv, d_v]      W  fp32 [L, H_r, H_s]
+ *   out   fp32 [L, n, H_r, d_v]
+ * and the batch is read as L copies of the sequences: sequence (l, s) = stacked sequence
+ * l * S + s at rows l * n + cu_seqlens[s]. Every other output is that of iamap_compress /
+ * iamap_mapped_av on the stacked batch (lse [H_s, L * n], mass [H_s, L * num_causal_blocks],
+ * the BSR index over L * num_rowblocks row blocks; iamap_layers_plan reports the stacked
+ * counts). Layer l of mapped_av mixes with W[l]. Workspace: iamap_layers_workspace_bytes with
+ * the stacked row-block count.
+ */
+int iamap_layers_plan(const int32_t* cu_seqlens_host, int num_seqs, int num_layers, int B,
+                      int64_t* num_rowblocks, int64_t* num_causal_blocks,
+                      int32_t* max_blocks_per_seq);
+size_t iamap_layers_workspace_bytes(int num_seqs, int num_layers, int64_t num_rowblocks);
+int iamap_compress_layers(const void* q, const void* k, const int32_t* cu_seqlens,
+                          const int32_t* cu_seqlens_host, int num_seqs, int64_t n,
+                          int num_layers, int H_s, int d, int B, float tau, int bias_window,
+                          float bias_value, float* lse, float* mass, uint64_t* headmask_dense,
+                          int32_t* row_ptr, int32_t* col_idx, uint64_t* headmask,
+                          int64_t* val_off, int64_t* counts, void* vals,
+                          int64_t vals_capacity_tiles, void* ws, size_t ws_bytes, void* stream);
+int iamap_mapped_av_layers(const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                           int num_seqs, int64_t n, int num_layers, int B, int H_s,
+                           const int32_t* row_ptr, const int32_t* col_idx,
+                           const uint64_t* headmask, const int64_t* val_off, const void* vals,
+                           int64_t vals_capacity_tiles, const float* W, int H_r, int H_kv,
+                           const void* v, int d_v, float* out, void* ws, size_t ws_bytes,
+                           void* stream);
 
 /*
  * Chunked prefill ("PKU MapFlow" news page, the paragraph on the vLLM integration: the fused

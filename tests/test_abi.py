@@ -230,3 +230,13 @@ def test_host_validation_of_chunk_and_sender_output(lib):
                                    fake, fake, fake, fake, 1, fake, 8, 3, fake, 64, fake, fake, 0,
                                    None)
     assert rc == -1 and "divide" in lib.iamap_last_error()
+
+
+def test_layers_plan_counts(lib):
+    """Several layers per launch: the stacked batch has num_layers copies of every sequence."""
+    one = lib.iamap_plan([0, 300, 370, 371], 3, 64)
+    assert lib.iamap_layers_plan([0, 300, 370, 371], 3, 4, 64) == (4 * one[0], 4 * one[1], one[2])
+    with pytest.raises(lib.IamapError):
+        lib.iamap_layers_plan([0, 300], 1, 0, 64)
+    assert lib.iamap_layers_workspace_bytes(3, 4, 4 * one[0]) > \
+        lib.iamap_compress_workspace_bytes(12, 4 * one[0])
