@@ -112,6 +112,7 @@ constexpr int kNGh = kNG / 2;    // pair slots of each readout group: even pairs
                                  // slots 0-1, odd pairs slots 2-3, so that every slot has one
                                  // consumer that takes its phases in order
 constexpr int kNV = 4;           // V tiles: one slot per receiver head of the CTA
+constexpr int kRecv = 2;         // exchange rounds in flight: receive buffers of 4 heads x 8 KB
 constexpr int kThreads = 608;    // 19 warps
 constexpr int kEpiWarps = 8;     // two readout groups of four warps
 constexpr int kMixCol = 256;     // first TMEM column of the mixing slots
@@ -120,8 +121,8 @@ constexpr uint32_t kTmemCols = 512;
 // barrier indices
 enum {
   P_FULL = 0, P_EMPTY = P_FULL + kMaxNP, W_FULL = P_EMPTY + kMaxNP, W_EMPTY = W_FULL + 2,
-  D_FULL = W_EMPTY + 2, D_EMPTY = D_FULL + kNG, RECV_FULL = D_EMPTY + kNG, BUF_FREE = RECV_FULL + 2,
-  V_FULL = BUF_FREE + 2, PV_DONE = V_FULL + kNV, O_FULL = PV_DONE + 2, MIX_DONE = O_FULL + 1,
+  D_FULL = W_EMPTY + 2, D_EMPTY = D_FULL + kNG, RECV_FULL = D_EMPTY + kNG, BUF_FREE = RECV_FULL + kRecv,
+  V_FULL = BUF_FREE + kRecv, PV_DONE = V_FULL + kNV, O_FULL = PV_DONE + 2, MIX_DONE = O_FULL + 1,
   NUM_BARS = MIX_DONE + 1
 };
 
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
     for (int i = 0; i < NUM_BARS; ++i) {
       uint32_t cnt = 1;
       if (i >= D_EMPTY && i < D_EMPTY + kNG) cnt = 4;
-      if (i >= BUF_FREE && i < BUF_FREE + 2) cnt = (uint32_t)C;
+      if (i >= BUF_FREE && i < BUF_FREE + kRecv) cnt = (uint32_t)C;
       tc::mbar_init(bar_addr(bars, i), cnt);
     }
     misc[1] = 0;
@@ -362,9 +363,9 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
       const uint32_t v_lbo = p.d_v == 128 ? 8192u : 0u;
       const uint16_t all_ctas = (uint16_t)((1u << C) - 1u);
       for (int t = 0; t < T; ++t) {
-        const int rs = t & 1;
+        const int rs = t % kRecv;
         tc::mbar_expect_tx(bar_addr(bars, RECV_FULL + rs), (uint32_t)G * 8192u);
-        tc::wait_bar(bar_addr(bars, RECV_FULL + rs), (t >> 1) & 1, abort_flag, p.status);
+        tc::wait_bar(bar_addr(bars, RECV_FULL + rs), (t / kRecv) & 1, abort_flag, p.status);
         tc::tc_fence_after();
         tc::fence_proxy_async_smem();  // peers' st.async data, read next by the tensor cores
         for (int rl = 0; rl < G; ++rl) {
@@ -379,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
             tc::mma_bf16(tmem + (uint32_t)rl * 64u, a, b, id_pv, (t > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        tc::mma_commit(bar_addr(bars, PV_DONE + rs));
+        tc::mma_commit(bar_addr(bars, PV_DONE + (t & 1)));
         tc::mma_commit_to_cluster(bar_addr(bars, BUF_FREE + rs), all_ctas);
       }
       tc::mma_commit(bar_addr(bars, O_FULL));
@@ -400,11 +401,11 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
     const bool releaser = (warp == 2 || warp == 13) && lane == 0;
     const int npg = (npair + 1 - eg) >> 1;   // pairs of this group per block
     for (int t = 0; t < T; ++t) {
-      const int ss = t & 1;
+      const int ss = t % kRecv;
       const int q = t * nch;          // this block's first chunk (global order)
       int gp = t * npg;               // its first pair within this group
-      // the receive buffers of round t-2 are free once every peer's P.V of that round completed
-      if (t >= 2) tc::wait_bar(bar_addr(bars, BUF_FREE + ss), ((t - 2) >> 1) & 1, abort_flag, p.status);
+      // the receive buffers of round t - kRecv are free once every peer's P.V of that round completed
+      if (t >= kRecv) tc::wait_bar(bar_addr(bars, BUF_FREE + ss), ((t - kRecv) / kRecv) & 1, abort_flag, p.status);
       const uint32_t recv_local = sbase + p.off_recv + (uint32_t)ss * (kG * 8192u);
       const uint32_t rbar_local = bar_addr(bars, RECV_FULL + ss);
       for (int cc = 2 * eg; cc < nch; cc += (cc & 1) ? 3 : 1) {
@@ -477,14 +478,14 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         }
       }
     }
-    // the last two exchange rounds: every peer's P.V commit has arrived here and every peer's copy
+    // the last kRecv exchange rounds: every peer's P.V commit has arrived here and every peer's copy
     // into this CTA has landed, so nothing remote targets this CTA's shared memory once it exits.
     // These waits ignore the abort flag (bounded at 200 ms each): after a timeout elsewhere the
     // other threads skip their waits, and a remote arrival must still not outlive the CTA.
     if (eg == 0)
-      for (int t = max(0, T - 2); t < T; ++t) {
-        tc::drain_bar(bar_addr(bars, BUF_FREE + (t & 1)), (t >> 1) & 1);
-        tc::drain_bar(bar_addr(bars, RECV_FULL + (t & 1)), (t >> 1) & 1);
+      for (int t = max(0, T - kRecv); t < T; ++t) {
+        tc::drain_bar(bar_addr(bars, BUF_FREE + t % kRecv), (t / kRecv) & 1);
+        tc::drain_bar(bar_addr(bars, RECV_FULL + t % kRecv), (t / kRecv) & 1);
       }
   }
 
@@ -517,7 +518,7 @@ int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream) {
   p.KH = (a.H_s + 15) / 16 * 16;
   p.RB = (a.H_s + 7) / 8 * 8;
   // everything but the sender ring, then as many ring slots as fit (at most kMaxNP)
-  const size_t fixed = (size_t)2 * p.NR * 128 + 1024 + (size_t)2 * kG * 8192 + (size_t)kNV * a.d_v * 128 +
+  const size_t fixed = (size_t)2 * p.NR * 128 + 1024 + (size_t)kRecv * kG * 8192 + (size_t)kNV * a.d_v * 128 +
                        (size_t)kEpiWarps * 2048 + sizeof(float) * (size_t)a.H_r * a.H_s + 8 * NUM_BARS + 96 + 4096;
   const size_t p_stage_b = (size_t)2 * p.RB * 128;
   const size_t budget = 232448 - 1024;
@@ -531,7 +532,7 @@ int mapped_av_tc_impl(const MappedAvArgs& a, cudaStream_t stream) {
   off += (size_t)2 * p.NR * 128;
   off = round_up(off, 1024);
   p.off_recv = (uint32_t)off;
-  off += (size_t)2 * kG * 8192;
+  off += (size_t)kRecv * kG * 8192;
   p.off_v = (uint32_t)off;
   off += (size_t)kNV * a.d_v * 128;
   p.off_scr = (uint32_t)off;
