@@ -102,8 +102,11 @@ constexpr int kMaxNP = 12;       // sender-slice ring: as many slots as shared m
 // A thread that issues TMA loads waits ~5 ns per 128-byte line of the box (measured on this B200:
 // 0.31 us for a 16 KB contiguous box, 0.49 us for a V tile spread over 64 tokens, i.e. 33-52 GB/s
 // per issuing thread, against ~130 GB/s per SM from L2 with four issuers), so the loads are
-// spread over several producer warps: four for the sender slices (chunks round-robin) and one
-// per receiver head for the V tiles (each a single 3-D box of both 64-dim halves).
+// spread over several producer warps: four for the sender slices and one per receiver head for
+// the V tiles (each a single 3-D box of both 64-dim halves). Ring slot s is always loaded by
+// producer warp s mod 4, so the uses of a slot are issued in order by one thread: a wait for the
+// release of use u - 1 never runs while use u - 2 is still pending (an mbarrier parity wait two
+// phases ahead would pass at once and let a load overwrite a slot still in use).
 constexpr int kPWarps = 4, kVWarps = 4;
 constexpr int kND = 8;           // mixing-result TMEM slots (chunks)
 constexpr int kNG = kND / 2;     // ... committed and released in pairs of chunks (one commit costs
@@ -229,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         const int k8 = (k + 7) >> 3;
         const int y0 = (int)(off * 64);   // first line of the block
         for (int c = 0; c < nch; ++c, ++q) {
-          if (q % kPWarps != pw) continue;
+          if ((q % NP) % kPWarps != pw) continue;   // slot q % NP is always loaded by one warp
           const int ps = q % NP;
           if (q >= NP) tc::wait_bar(bar_addr(bars, P_EMPTY + ps), ((q / NP) - 1) & 1, abort_flag, p.status);
           tc::mbar_expect_tx(bar_addr(bars, P_FULL + ps), 2u * (uint32_t)k8 * 8u * 128u);
@@ -243,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
       // drain: the final load of every slot, where this warp issued it, has landed (earlier uses
       // of a slot are two phases back and must not be waited on)
       for (int qq = max(0, q - NP); qq < q; ++qq)
-        if (qq % kPWarps == pw) tc::drain_bar(bar_addr(bars, P_FULL + qq % NP), (qq / NP) & 1);
+        if ((qq % NP) % kPWarps == pw) tc::drain_bar(bar_addr(bars, P_FULL + qq % NP), (qq / NP) & 1);
     }
   } else if (warp == 7) {
     // ------------------------------ W' of each stored block ------------------------------
