@@ -411,53 +411,57 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
       if (t >= kRecv) tc::wait_bar(bar_addr(bars, BUF_FREE + ss), ((t - kRecv) / kRecv) & 1, abort_flag, p.status);
       const uint32_t recv_local = sbase + p.off_recv + (uint32_t)ss * (kG * 8192u);
       const uint32_t rbar_local = bar_addr(bars, RECV_FULL + ss);
-      for (int cc = 2 * eg; cc < nch; cc += (cc & 1) ? 3 : 1) {
-        const int gs = eg * kNGh + gp % kNGh, j = cc & 1;
-        const int ch = c0 + cc;
-        if (j == 0) {
-          tc::wait_bar(bar_addr(bars, D_FULL + gs), (gp / kNGh) & 1, abort_flag, p.status);
-          // the pair's mixing MMAs completed: their sender slots can be refilled
-          if (releaser)
-            for (int jj = 0; jj < min(2, nch - cc); ++jj) tc::mbar_arrive(bar_addr(bars, P_EMPTY + (q + cc + jj) % NP));
-        }
+      for (int cc = 2 * eg; cc < nch; cc += 4) {
+        // one pair of chunks (cc, cc + 1): both TMEM loads before one wait
+        const int gs = eg * kNGh + gp % kNGh;
+        const int nj = min(2, nch - cc);
+        tc::wait_bar(bar_addr(bars, D_FULL + gs), (gp / kNGh) & 1, abort_flag, p.status);
+        // the pair's mixing MMAs completed: their sender slots can be refilled
+        if (releaser)
+          for (int jj = 0; jj < nj; ++jj) tc::mbar_arrive(bar_addr(bars, P_EMPTY + (q + cc + jj) % NP));
         tc::tc_fence_after();
-        uint32_t v[32];
-        const uint32_t ta = tmem + lane_base + (uint32_t)kMixCol + (uint32_t)(2 * gs + j) * (uint32_t)p.NR;
+        uint32_t v[2][32];
+        const uint32_t ta = tmem + lane_base + (uint32_t)kMixCol + (uint32_t)(2 * gs) * (uint32_t)p.NR;
         if (p.NR == 32) {
-          IAMAP_TMEM_LD32(ta, v);
+          IAMAP_TMEM_LD32(ta, v[0]);
+          if (nj == 2) IAMAP_TMEM_LD32(ta + 32u, v[1]);
         } else {
-          IAMAP_TMEM_LD16(ta, v);
+          IAMAP_TMEM_LD16(ta, v[0]);
+          if (nj == 2) IAMAP_TMEM_LD16(ta + 16u, v[1]);
 #pragma unroll
-          for (int i = 16; i < 32; ++i) v[i] = 0u;
+          for (int i = 16; i < 32; ++i) v[0][i] = v[1][i] = 0u;
         }
         tc::tmem_ld_wait();
-        if (j == 1 || cc + 1 == nch) {
-          tc::tc_fence_before();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar_addr(bars, D_EMPTY + gs));
+        ++gp;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (j >= nj) break;
+          const int ch = c0 + cc + j;
+          // transpose: position = lane, head = register  ->  16-byte runs of one head
+#pragma unroll
+          for (int r = 0; r < 32; ++r)
+            if (r < p.NR)
+              reinterpret_cast<__nv_bfloat16*>(scr)[r * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[j][r]));
           __syncwarp();
-          if (lane == 0) tc::mbar_arrive(bar_addr(bars, D_EMPTY + gs));
-          ++gp;
-        }
-        // transpose: position = lane, head = register  ->  16-byte runs of one head
+          const int pos0 = 32 * e;                          // this warp's first position in the chunk
+          const int arow = 2 * ch + (pos0 >> 6);            // tile row
+          const int jc = ((pos0 & 63) >> 3) + o;            // 16-byte chunk of the row
+          const uint32_t row_off = (uint32_t)arow * 128u + ((uint32_t)(jc ^ (arow & 7)) << 4);
 #pragma unroll
-        for (int r = 0; r < 32; ++r)
-          if (r < p.NR)
-            reinterpret_cast<__nv_bfloat16*>(scr)[r * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[r]));
-        __syncwarp();
-        const int pos0 = 32 * e;                          // this warp's first position in the chunk
-        const int arow = 2 * ch + (pos0 >> 6);            // tile row
-        const int jc = ((pos0 & 63) >> 3) + o;            // 16-byte chunk of the row
-        const uint32_t row_off = (uint32_t)arow * 128u + ((uint32_t)(jc ^ (arow & 7)) << 4);
-#pragma unroll
-        for (int vv = 0; vv < 4; ++vv) {
-          const int r = 8 * vv + rq;
-          if (r < p.H_r) {
-            const uint4 val = *reinterpret_cast<const uint4*>(scr + r * 64 + o * 16);
-            const uint32_t c2 = (uint32_t)(r >> 2);
-            const uint32_t dst = tc::map_to_cta(recv_local + (uint32_t)(r & 3) * 8192u + row_off, c2);
-            tc::st_async_v4(dst, val, tc::map_to_cta(rbar_local, c2));
+          for (int vv = 0; vv < 4; ++vv) {
+            const int r = 8 * vv + rq;
+            if (r < p.H_r) {
+              const uint4 val = *reinterpret_cast<const uint4*>(scr + r * 64 + o * 16);
+              const uint32_t c2 = (uint32_t)(r >> 2);
+              const uint32_t dst = tc::map_to_cta(recv_local + (uint32_t)(r & 3) * 8192u + row_off, c2);
+              tc::st_async_v4(dst, val, tc::map_to_cta(rbar_local, c2));
+            }
           }
+          __syncwarp();
         }
-        __syncwarp();
       }
     }
     // output rows (first group): TMEM lane = d_v index, column = rl * 64 + row of the block
