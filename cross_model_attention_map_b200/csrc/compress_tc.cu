@@ -6,12 +6,14 @@
 // pair of row blocks (I0 = 2P, I1 = 2P + 1: 128 query rows, one per TMEM lane) of one sender head.
 //
 // Stage 1 (stats_tc_kernel): S = Q K^T for 128 keys at a time (column blocks 2T, 2T + 1) lands in
-// one of two 128-column TMEM buffers. Eight softmax warps read it back, one thread per (row,
-// column block): the block's log2-sum c_iJ = log2 sum_j 2^(s_ij log2(e)/sqrt(d)) is kept in TMEM
-// column 256 + J, and the row's running log-sum-exp in registers. Afterwards the same threads
-// form lse_i, the block masses sum_i 2^(c_iJ - lse_i) (a 32 x 32 butterfly per warp sums over
-// rows), and the cumulative-mass choice of each row block. Rows with more than 256 column blocks
-// (sequences longer than 16384 tokens) take the mma.sync kernel instead.
+// one of two 128-column TMEM buffers (tile T in buffer T % 2). Sixteen softmax warps, four per SM
+// sub-partition, read it back, one thread per (row, column block): the warps of even tiles and
+// those of odd tiles run side by side, so that the exponentials of one set overlap the waits of
+// the other. The block's log2-sum c_iJ = log2 sum_j 2^(s_ij log2(e)/sqrt(d)) is kept in TMEM
+// column 256 + J. Afterwards the same threads form lse_i from the c values, the block masses
+// sum_i 2^(c_iJ - lse_i) (a 32 x 32 butterfly per warp sums over rows), and the cumulative-mass
+// choice of each row block. Rows with more than 256 column blocks (sequences longer than 16384
+// tokens) take the mma.sync kernel instead.
 //
 // Stage 2 (extract_tc_kernel): for every column block J that this head keeps in I0 or I1,
 // S = Q K_J^T (128 x 64) is recomputed into TMEM; two groups of four warps take alternate blocks
@@ -19,11 +21,14 @@
 // that each 128-byte tile row leaves as one coalesced run (rows of the k present heads of a
 // stored block are interleaved: row i of head rank t is line i * k + t of the block).
 //
-// Roles (320 threads): warps 0-7 softmax / writers, warp 8 TMA producer, warp 9 MMA issuer (and
-// TMEM owner). Every wait is bounded (2 s; then IAMAP_DEV_TIMEOUT and an orderly exit).
+// Roles: stats (576 threads) warps 0-15 softmax, warp 16 TMA producer (lanes 0 and 1: the two
+// 64-dim panels of each key tile), warp 17 MMA issuer and TMEM owner; extract (320 threads)
+// warps 0-7 writers, warp 8 TMA producer, warp 9 MMA issuer and TMEM owner. Every wait is bounded
+// (2 s; then IAMAP_DEV_TIMEOUT and an orderly exit).
 #include <algorithm>
 
 #include "tc_utils.cuh"
+#include "exp2_fma.cuh"
 #include "internal.h"
 
 namespace iamap {
@@ -31,8 +36,9 @@ namespace tccomp {
 
 constexpr int kRows = 128;         // query rows per CTA (row blocks 2P, 2P + 1)
 constexpr int kThreads = 320;      // extract: warps 0-7 writers, 8 TMA, 9 MMA
-constexpr int kSThreads = 352;     // stats: warps 0-7 softmax, 8 and 10 TMA, 9 MMA
-constexpr int kSoft = 256;         // softmax threads
+constexpr int kSThreads = 576;     // stats: warps 0-15 softmax, 16 TMA, 17 MMA
+constexpr int kSMmaWarp = 17;
+constexpr int kSoft = 512;         // stats: softmax threads
 constexpr int kSStages = 4;        // stats: key-tile ring (128 keys per tile)
 constexpr int kXStages = 2;        // extract: key-tile ring (64 keys per tile)
 constexpr int kCCol = 256;         // stats: TMEM column of c_i0
@@ -160,26 +166,32 @@ __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-// c = log2 of sum_j 2^(x_j) over one thread's 64 logits of column block J (keys j0 .. j0 + 63) of
-// row i, x_j = s_j * sc (+ bias_log2 where 0 <= i - j < bias_window), x_j = -inf above the
-// diagonal. `plain`: J is below the row's block, so there is no mask, and the bias is checked.
-// The masked path overwrites v with the x_j.
-__device__ __forceinline__ float block_log2sum(uint32_t (&v)[64], int i, int j0, bool plain,
-                                               float sc, int bias_window, float bias_log2) {
-  if (plain && !(bias_window > 0 && i - j0 - 63 < bias_window)) {
-    float m8[8];
+// One thread's 64 logits of column block J (keys j0 .. j0 + 63) of row i: x_j = s_j * sc
+// (+ bias_log2 where 0 <= i - j < bias_window), x_j = -inf above the diagonal. The block's
+// log2-sum c = log2 sum_j 2^(x_j) = m + log2 sum_j 2^(x_j - m) with m = max_j x_j is taken in two
+// passes, the max and then the exponentials, so that other work can sit between them.
+
+// A block with every key present and no bias: max of the raw scores (3-input max).
+__device__ __forceinline__ float raw_max64(const uint32_t (&v)[64]) {
+  float m[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(v[k]);
+  for (int k = 0; k < 4; ++k) m[k] = fmaxf(__uint_as_float(v[k]), __uint_as_float(v[k + 4]));
 #pragma unroll
-    for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(v[e]));
-    const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-    const float nm = -mx * sc;
-    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int e = 8; e < 64; e += 8) {
 #pragma unroll
-    for (int e = 0; e < 64; ++e) s4[e & 3] += ex2(fmaf(__uint_as_float(v[e]), sc, nm));
-    return mx * sc + lg2((s4[0] + s4[1]) + (s4[2] + s4[3]));
+    for (int k = 0; k < 4; ++k) {
+      const float a = __uint_as_float(v[e + k]), b = __uint_as_float(v[e + 4 + k]);
+      asm("max.f32 %0, %0, %1, %2;" : "+f"(m[k]) : "f"(a), "f"(b));
+    }
   }
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m[0]), "f"(m[1]), "f"(fmaxf(m[2], m[3])));
+  return r;
+}
+
+// Any other block: the x_j replace v (scaled, biased, masked); returns their max.
+__device__ __forceinline__ float masked_max64(uint32_t (&v)[64], int i, int j0, float sc,
+                                              int bias_window, float bias_log2) {
   float m8[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
@@ -192,13 +204,55 @@ __device__ __forceinline__ float block_log2sum(uint32_t (&v)[64], int i, int j0,
     v[e] = __float_as_uint(y);
     m8[e & 7] = fmaxf(m8[e & 7], y);
   }
-  const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-  if (mx == -INFINITY) return -INFINITY;
+  return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+}
+
+// Number of the 32 column pairs of a plain block whose exponentials run on the FMA pipe
+// (exp2_fma.cuh); the rest use ex2 on the MUFU unit. 0 by default: on a B200, prefill8k stats
+// took 0.44 ms with 0 pairs, 0.45 with 8, 0.46 with 12 and 0.50 with 16 (at 1965 MHz), since the
+// MUFU unit is not this loop's only limit and the polynomial costs more issue slots than it frees.
+#ifndef IAMAP_STATS_FMA_PAIRS
+#define IAMAP_STATS_FMA_PAIRS 0
+#endif
+constexpr int kFmaPairs = IAMAP_STATS_FMA_PAIRS;
+
+__device__ __forceinline__ constexpr bool fma_pair(int q) {
+  return (q * kFmaPairs) % 32 < kFmaPairs;   // spread evenly over the block
+}
+
+// sum_j 2^(s_j * sc + nm) over a plain block (nm = -max_j s_j * sc), packed pairs.
+__device__ __forceinline__ float plain_exp2_sum64(const uint32_t (&v)[64], float sc, float nm) {
+  const uint64_t sc2 = f2_splat(sc), nm2 = f2_splat(nm);
+  uint64_t acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = f2_splat(0.f);
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1])),
+                              sc2, nm2);
+    uint64_t e;
+    if (fma_pair(q)) {
+      e = exp2_fma_x2(x);
+    } else {
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      e = f2_pack(ex2(x0), ex2(x1));
+    }
+    acc[q & 3] = f2_add(acc[q & 3], e);
+  }
+  const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  float a, b;
+  f2_unpack(t, a, b);
+  return a + b;
+}
+
+// sum_j 2^(x_j - m) over a block whose x_j are in v (masked_max64), m > -inf.
+__device__ __forceinline__ float masked_exp2_sum64(const uint32_t (&v)[64], float m) {
   float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int e = 0; e < 64; ++e) s4[e & 3] += ex2(__uint_as_float(v[e]) - mx);
-  return mx + lg2((s4[0] + s4[1]) + (s4[2] + s4[3]));
+  for (int e = 0; e < 64; ++e) s4[e & 3] += ex2(__uint_as_float(v[e]) - m);
+  return (s4[0] + s4[1]) + (s4[2] + s4[3]);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -215,9 +269,9 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase, sK = sbase + kQBytes;
   float* aux = reinterpret_cast<float*>(smem + kQBytes + kSStages * kKStage);
-  float* ml_m = aux;                  // [2][128] running max (log2) of each group
-  float* ml_l = ml_m + 2 * kRows;     // [2][128] running sum
-  float* lse_s = ml_l + 2 * kRows;    // [128] row lse (log2)
+  float* ml_m = aux;                  // [4][128] max (log2) of each softmax group's c values
+  float* ml_l = ml_m + 4 * kRows;     // [4][128] their sums of exponentials
+  float* lse_s = ml_l + 4 * kRows;    // [128] row lse (log2)
   float* part = lse_s + kRows;        // [4][256] per-quarter column sums
   float* mass_s = part + 4 * kMaxNb;  // [2][256]
   float* sorted_s = mass_s + 2 * kMaxNb;
@@ -248,18 +302,18 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
     misc[1] = 0;
     tc::fence_barrier_init();
   }
-  if (warp == 9) tc::tmem_alloc(smem_u32(misc), 512);
+  if (warp == kSMmaWarp) tc::tmem_alloc(smem_u32(misc), 512);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  if (warp == 8 || warp == 10) {
+  if (warp == kSMmaWarp - 1) {
     // ------------------------------ TMA: Q once, then the key tiles ------------------------------
     // One thread issues a 16 KB box only every ~0.3 us, so the two 64-dim panels of each key tile
-    // come from two warps (warp 8: panel 0 and Q, warp 10: panel 1), each arriving on K_FULL.
-    const int pan = warp == 8 ? 0 : 1;
-    if (lane == 0 && pan < NPAN) {
+    // come from two lanes (lane 0: panel 0 and Q, lane 1: panel 1), each arriving on K_FULL.
+    const int pan = lane;
+    if (pan < NPAN) {
       if (pan == 0) {
         tc::prefetch_tmap(&p.q_map);
         tc::mbar_expect_tx(bar_addr(bars, Q_FULL), kQBytes);
@@ -281,7 +335,7 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
         tc::drain_bar(bar_addr(bars, K_FULL + T % kSStages), (T / kSStages) & 1);
       if (pan == 0) tc::drain_bar(bar_addr(bars, Q_FULL), 0);
     }
-  } else if (warp == 9) {
+  } else if (warp == kSMmaWarp) {
     // ------------------------------ MMA: S_b = Q K_T^T (128 x 128, fp32 in TMEM) ----------------
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 0);
@@ -305,74 +359,90 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
     }
   } else {
     // ------------------------------ softmax: one thread per (row, column block) -----------------
-    const int qd = warp & 3, g = warp >> 2;
+    // 16 warps, four per SM sub-partition: the warp's lane quarter qd gives its 32 rows, g the
+    // column block 2T + g of a tile and tp the tiles it takes (T % 2 == tp, TMEM buffer tp). The
+    // two tile parities run side by side, so one warp's waits (TMEM load, barriers, dependent
+    // arithmetic) overlap the other warps' exponentials.
+    const int qd = warp & 3, grp = warp >> 2, g = grp & 1, tp = grp >> 1;
     const int r = 32 * qd + lane;                 // TMEM lane = pair-local row
     const int Ir = I0 + (r >> 6);                 // row block (uniform over the warp)
     const int i = kRows * P + r;                  // sequence-local row
     const bool valid = i < L && Ir >= Ifirst;
     const uint32_t t_lane = (uint32_t)(32 * qd) << 16;
     const float sc = p.scale_log2;
-    float m_acc = -INFINITY, l_acc = 0.f;
-    // The TMEM load of tile T + 1 is issued before the exponentials of tile T, so that its latency
-    // hides behind them (two register sets, the loop unrolled by two).
-    uint32_t va[64], vb[64];
-    auto issue = [&](uint32_t (&v)[64], int T) {
-      if (2 * T + g <= Ir) {
-        const uint32_t col = (uint32_t)((T & 1) * 128 + g * 64);
+    uint32_t v[64];
+    for (int T = tp; T < nT; T += 2) {
+      const int J = 2 * T + g;
+      const bool has = J <= Ir;
+      tc::wait_bar(bar_addr(bars, S_FULL + tp), (T >> 1) & 1, abort_flag, p.status);
+      tc::tc_fence_after();
+      if (has) {
+        const uint32_t col = (uint32_t)(tp * 128 + g * 64);
         IAMAP_TMEM_LD32(tmem + t_lane + col, v);
         IAMAP_TMEM_LD32(tmem + t_lane + col + 32u, (v + 32));
+        tc::tmem_ld_wait();
       }
-    };
-    auto step = [&](uint32_t (&cur)[64], uint32_t (&nxt)[64], int T) {
-      const int J = 2 * T + g;
-      if (J <= Ir) tc::tmem_ld_wait();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar_addr(bars, S_EMPTY + (T & 1)));
-      bool early = false;
-      if (T + 1 < nT && tc::mbar_try_wait(bar_addr(bars, S_FULL + ((T + 1) & 1)), ((T + 1) >> 1) & 1)) {
-        tc::tc_fence_after();
-        issue(nxt, T + 1);
-        early = true;
-      }
-      if (J <= Ir) {
-        const float c = block_log2sum(cur, i, 64 * J, J < Ir, sc, p.bias_window, p.bias_log2);
-        if (c > m_acc) {
-          l_acc = l_acc * ex2(m_acc - c) + 1.f;
-          m_acc = c;
-        } else if (c > -INFINITY) {
-          l_acc += ex2(c - m_acc);
+      if (lane == 0) tc::mbar_arrive(bar_addr(bars, S_EMPTY + tp));
+      if (has) {
+        float c;
+        if (J < Ir && !(p.bias_window > 0 && i - 64 * J - 63 < p.bias_window)) {
+          const float m = raw_max64(v) * sc;
+          c = m + lg2(plain_exp2_sum64(v, sc, -m));
+        } else {
+          const float m = masked_max64(v, i, 64 * J, sc, p.bias_window, p.bias_log2);
+          c = m == -INFINITY ? -INFINITY : m + lg2(masked_exp2_sum64(v, m));
         }
         tmem_st1(tmem + t_lane + (uint32_t)(kCCol + J), c);
       }
-      if (T + 1 < nT && !early) {
-        tc::wait_bar(bar_addr(bars, S_FULL + ((T + 1) & 1)), ((T + 1) >> 1) & 1, abort_flag, p.status);
-        tc::tc_fence_after();
-        issue(nxt, T + 1);
-      }
-    };
-    if (nT > 0) {
-      tc::wait_bar(bar_addr(bars, S_FULL), 0, abort_flag, p.status);
-      tc::tc_fence_after();
-      issue(va, 0);
-    }
-    for (int T = 0; T < nT; T += 2) {
-      step(va, vb, T);
-      if (T + 1 < nT) step(vb, va, T + 1);
     }
     tmem_st_wait();
-
-    // ---- row log-sum-exp (both groups' partial sums) ----
-    ml_m[g * kRows + r] = m_acc;
-    ml_l[g * kRows + r] = l_acc;
     tc::tc_fence_before();
     tc::named_bar(1, kSoft);
     tc::tc_fence_after();
-    if (g == 0) {
-      const float m0 = ml_m[r], m1 = ml_m[kRows + r];
-      const float m = fmaxf(m0, m1);
+
+    // ---- row log-sum-exp from the row's c values: group grp takes the 32-column chunks
+    // ch = grp mod 4, then the four partial (max, sum) pairs are combined ----
+    const int nJ = min(2 * P + 2, nb);
+    {
+      float m_acc = -INFINITY, l_acc = 0.f;
+      for (int ch = grp; ch * 32 < nJ; ch += 4) {
+        uint32_t cv[32];
+        IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(kCCol + 32 * ch), cv);
+        tc::tmem_ld_wait();
+        float cm = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (32 * ch + e <= Ir) cm = fmaxf(cm, __uint_as_float(cv[e]));
+        if (cm > -INFINITY) {
+          float cs = 0.f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (32 * ch + e <= Ir) cs += ex2(__uint_as_float(cv[e]) - cm);
+          if (cm > m_acc) {
+            l_acc = l_acc * ex2(m_acc - cm) + cs;
+            m_acc = cm;
+          } else {
+            l_acc += cs * ex2(cm - m_acc);
+          }
+        }
+      }
+      ml_m[grp * kRows + r] = m_acc;
+      ml_l[grp * kRows + r] = l_acc;
+    }
+    tc::named_bar(1, kSoft);
+    if (grp == 0) {
+      float m = ml_m[r];
+#pragma unroll
+      for (int k = 1; k < 4; ++k) m = fmaxf(m, ml_m[k * kRows + r]);
       float lse2 = -INFINITY;
-      if (m > -INFINITY) lse2 = m + lg2(ml_l[r] * ex2(m0 - m) + ml_l[kRows + r] * ex2(m1 - m));
+      if (m > -INFINITY) {
+        float l = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) l += ml_l[k * kRows + r] * ex2(ml_m[k * kRows + r] - m);
+        lse2 = m + lg2(l);
+      }
       lse_s[r] = lse2;
       if (valid) p.lse[(int64_t)h * p.n + row0 + i] = lse2 * kLn2;
     }
@@ -380,9 +450,8 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
     if (p.mass != nullptr) {
 
     // ---- block masses: sum over the valid rows of 2^(c_iJ - lse_i) ----
-    const int nJ = min(2 * P + 2, nb);
     const float lr = lse_s[r];
-    for (int ch = g; ch * 32 < nJ; ch += 2) {
+    for (int ch = grp; ch * 32 < nJ; ch += 4) {
       uint32_t cv[32];
       IAMAP_TMEM_LD32(tmem + t_lane + (uint32_t)(kCCol + 32 * ch), cv);
       tc::tmem_ld_wait();
@@ -448,7 +517,7 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kSMmaWarp) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, 512);
   }
@@ -802,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
 template <int D>
 static size_t stats_smem() {
   return 1024 + (size_t)(D / 64) * kPanel128 * (1 + kSStages) +
-         sizeof(float) * (2 * kRows + 2 * kRows + kRows + 4 * kMaxNb + 2 * kMaxNb + 2 * kMaxNb) +
+         sizeof(float) * (4 * kRows + 4 * kRows + kRows + 4 * kMaxNb + 2 * kMaxNb + 2 * kMaxNb) +
          sizeof(int) * 2 * kMaxNb + 8 * NUM_BARS + 16;
 }
 template <int D, bool OUT>

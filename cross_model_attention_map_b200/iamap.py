@@ -71,6 +71,7 @@ _SIGS = {
                                      _P, _SZ, _P]),
     "iamap_mapping_consistency": (_I, [_P, _P, _I, _P, _P]),
     "iamap_selftest_wait_timeout": (_I, [_I, _P, _P]),
+    "iamap_selftest_exp2": (_I, [_P, _P, _P, _I64, _P]),
     "iamap_prefix_num_keys": (_I, [_P, _I, _I, ctypes.POINTER(_I64)]),
     "iamap_bsr_check_host": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I64,
                                   ctypes.POINTER(_I64)]),
@@ -442,6 +443,11 @@ def iamap_head_match_metric(q_small, k_small, L_s, H_small, d_small, q_large, k_
 def iamap_selftest_wait_timeout(limit_us, gave_up, stream=None):
     _check("iamap_selftest_wait_timeout", _lib.iamap_selftest_wait_timeout(
         limit_us, _ptr(gave_up), _stream(stream)))
+
+
+def iamap_selftest_exp2(x, y_fma, y_mufu, n, stream=None):
+    _check("iamap_selftest_exp2", _lib.iamap_selftest_exp2(
+        _ptr(x), _ptr(y_fma), _ptr(y_mufu), n, _stream(stream)))
 
 
 def iamap_mapping_consistency(a, b, n_heads, agree, stream=None):

@@ -36,6 +36,8 @@
  *                lookup of a prompt's blocks and of its longest cached prefix. (MapFlow news
  *                page, storage-and-execution part, second component.)
  *   iamap_selftest_wait_timeout  exercises the bounded-wait failure path on the GPU.
+ *   iamap_selftest_exp2  evaluates the FMA-pipe exponential that the compress kernels can use
+ *                beside the MUFU one, for accuracy tests.
  *
  * Conventions (all entry points):
  *   - Return 0 (IAMAP_OK) or a negative IAMAP_ERR_* code; iamap_last_error() gives a
@@ -432,6 +434,15 @@ int iamap_mapped_av_paged_noalloc(const float* p_rows, int ctx_stride, const flo
  * context stays usable. Asynchronous on stream.
  */
 int iamap_selftest_wait_timeout(int limit_us, int* gave_up, void* stream);
+
+/*
+ * Exponential self-test: y_fma[k] = 2^x[k] by the FMA-pipe method of the compress kernels (exact
+ * base-2 argument reduction 2^x = 2^n 2^f, n = rint(x), then a degree-5 minimax polynomial for
+ * 2^f on [-1/2, 1/2]; inputs below -126 give 2^-126) and y_mufu[k] = 2^x[k] by ex2.approx.ftz on
+ * the MUFU unit, for n elements (device fp32 arrays, n >= 0; elements are evaluated in pairs as
+ * in the kernels). Meant for x <= 0, the range the softmax passes use. Asynchronous on stream.
+ */
+int iamap_selftest_exp2(const float* x, float* y_fma, float* y_mufu, int64_t n, void* stream);
 
 /*
  * Head matching (calibration). q_small / k_small bf16 [L_s, n, H_small, d_small];
