@@ -96,11 +96,13 @@ struct ExtractParams {
   __nv_bfloat16* vals;
   int64_t capacity;
   unsigned int* status;
-  // dense mode (head_match maps): every causal tile of every head, head-major, row-major tiles
-  // (tile I(I+1)/2 + J of head (s * H_s + h) at index (s * H_s + h) * dense_tiles + ...), with the
+  // dense mode (head_match maps): every causal tile of every head, chunk-major: row r of tile
+  // t = I(I+1)/2 + J of head hh = s * H_s + h is the 128-byte line (t * 64 + r) * dense_heads + hh,
+  // so that one 64-element chunk of the flattened maps of all heads is contiguous; with the
   // sum and the squared norm of each head's rounded map added into sum1 / norm2
   int dense;
   int64_t dense_tiles;
+  int dense_heads;
   float* norm2;
   float* sum1;
   // sender output (extract_tc_kernel<D, true>): V_s bf16 viewed {64, n_k, H_s * d_vs / 64}, box
@@ -550,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
   unsigned char* stage_all = smem + kQBytes + kXStages * kKStage + (OUT ? kVStages * kVStage : 0);
   // 8 warps x 4 KB per staging buffer
   int64_t* base_s = reinterpret_cast<int64_t*>(stage_all + kStageBufs * 8 * 4096);   // [2][256]
-  int* rk_s = reinterpret_cast<int*>(base_s + 2 * kMaxNb);               // [2][256] rank | k << 8
+  int* rk_s = reinterpret_cast<int*>(base_s + 2 * kMaxNb);               // [2][256] rank | k << 16
   int* ulist = rk_s + 2 * kMaxNb;                                        // [256] union of J
   uint64_t* bar_mem = reinterpret_cast<uint64_t*>(ulist + kMaxNb);
   uint32_t* misc = reinterpret_cast<uint32_t*>(bar_mem + kBars);         // [0] tmem [1] abort [2] count
@@ -588,8 +590,9 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
     for (int idx = tid; idx < 2 * kMaxNb; idx += kThreads) {
       const int k = idx / kMaxNb, J = idx - k * kMaxNb, I = I0 + k;
       if (I < nb && J <= I) {
-        base_s[idx] = ((int64_t)s * p.H_s + h) * p.dense_tiles + (int64_t)I * (I + 1) / 2 + J;
-        rk_s[idx] = 1 << 8;
+        // the tile's rows are lines of a "block" of dense_heads interleaved heads (rank hh)
+        base_s[idx] = ((int64_t)I * (I + 1) / 2 + J) * p.dense_heads;
+        rk_s[idx] = (s * p.H_s + h) | (p.dense_heads << 16);
       }
     }
   } else if (warp < 2 && I0 + warp < nb && I0 + warp >= Ifirst) {
@@ -601,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
       if ((m >> h) & 1ull) {
         const int J = p.col_idx[u];
         base_s[warp * kMaxNb + J] = p.val_off[u];
-        rk_s[warp * kMaxNb + J] = __popcll(m & below) | (__popcll(m) << 8);
+        rk_s[warp * kMaxNb + J] = __popcll(m & below) | (__popcll(m) << 16);
       }
     }
   }
@@ -733,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
       const int J = ulist[t];
       const int64_t base = base_s[kb * kMaxNb + J];
       const int rk = rk_s[kb * kMaxNb + J];
-      const int rank = rk & 255, k = rk >> 8;
+      const int rank = rk & 0xffff, k = rk >> 16;
       // OUT: every block feeds the P.V MMA, so every block's P is staged
       const bool stage = OUT || base >= 0;
       if (stage) {
@@ -939,6 +942,7 @@ int compress_extract_tc_launch(const CompressArgs& a, cudaStream_t stream) {
   p.tok0 = a.tok0;
   p.dense = a.dense;
   p.dense_tiles = a.dense_tiles;
+  p.dense_heads = a.dense && a.dense_tiles > 0 ? (int)(a.capacity / a.dense_tiles) : 0;
   p.norm2 = a.norm2;
   p.sum1 = a.sum1;
   p.tab = a.tab;

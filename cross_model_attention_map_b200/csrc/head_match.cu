@@ -4,13 +4,16 @@
 // small-model head; prompts longer than tau_t are truncated).
 //
 // 1. maps_kernel<D>: one CTA per (head, row block) computes the causal softmax map rows of the
-//    first n_used tokens (two sweeps over the key tiles: row log-sum-exp, then probabilities) and
-//    writes them as bf16 64 x 64 tiles in causal-block order, zeros above the diagonal and past
-//    n_used. The flattened map of a head is its run of tiles. The squared norm of the bf16 map is
-//    accumulated alongside.
+//    first n_used tokens (two sweeps over the key tiles: row log-sum-exp, then probabilities) as
+//    bf16 64 x 64 tiles in causal-block order, zeros above the diagonal and past n_used. The
+//    flattened map of a head is its tiles' rows in order: 64-element chunks c = tile * 64 + row.
+//    The maps of all heads are stored chunk-major (chunk c of head hh is the 128-byte line
+//    c * heads + hh), so that the Gram reads each chunk of 128 heads as one contiguous 16 KB run.
+//    The squared norm and the sum of the bf16 map are accumulated alongside. (Prompts of 2048+
+//    tokens take the tcgen05 compress kernels instead, which write the same layout.)
 // 2. gram_tc_kernel: C_raw = A_large . A_small^T over the flattened maps on the tcgen05 tensor
-//    cores (split-K; operands by TMA with 128-byte swizzle, fp32 accumulator in TMEM, atomic fp32
-//    reduction of the K splits).
+//    cores (split-K; operands by TMA with 128-byte swizzle from the chunk-major maps viewed
+//    {64, heads, chunks}, fp32 accumulator in TMEM, atomic fp32 reduction of the K splits).
 // 3. finalize_kernel: the similarity of every (large, small) pair from C_raw and each map's sum and
 //    squared norm, and the argmax per large head (lowest small-head index on ties). The method
 //    section of the IAM notes compares cosine similarity, Minkowski distance and the Pearson
@@ -97,7 +100,8 @@ __global__ void __launch_bounds__(kTileThreads) maps_kernel(MapsParams p) {
   const float lB = m_run[1] + lg2(l_run[1]);
 
   // Sweep 2: probabilities as bf16 tiles; squared norm of the rounded values.
-  __nv_bfloat16* out = p.maps + ((int64_t)head * p.tiles + (int64_t)I * (I + 1) / 2) * kTile * kTile;
+  // chunk-major: row r of tile t of this head is line (t * 64 + r) * heads + head
+  __nv_bfloat16* out = p.maps + ((int64_t)I * (I + 1) / 2 * kTile * heads + head) * kTile;
   float nrm = 0.f, tot = 0.f;
   load_k_tile<D>(sK0, kb, rs, 0, L, tid);
   cp_async_commit();
@@ -122,10 +126,11 @@ __global__ void __launch_bounds__(kTileThreads) maps_kernel(MapsParams p) {
       *reinterpret_cast<uint32_t*>(stage + rB * kTile + ((nt ^ (rB & 7)) << 3) + 2 * t4) = wb;
     }
     __syncthreads();
-    uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)J * kTile * kTile);
+    __nv_bfloat16* dst = out + (int64_t)J * kTile * heads * kTile;
     for (int c = tid; c < kTile * 8; c += kTileThreads) {
       const int r = c >> 3, ch = c & 7;
-      dst[c] = *reinterpret_cast<const uint4*>(stage + r * kTile + ((ch ^ (r & 7)) << 3));
+      *reinterpret_cast<uint4*>(dst + (int64_t)r * heads * kTile + ch * 8) =
+          *reinterpret_cast<const uint4*>(stage + r * kTile + ((ch ^ (r & 7)) << 3));
     }
   }
 #pragma unroll
@@ -153,8 +158,8 @@ __global__ void __launch_bounds__(kTileThreads) maps_kernel(MapsParams p) {
 constexpr int kGtStages = 5, kGtThreads = 192;
 
 struct GramTcParams {
-  CUtensorMap a_map;   // maps_large viewed [M][K] bf16, box {64, 128}
-  CUtensorMap b_map;   // maps_small viewed [N][K] bf16, box {64, BN}
+  CUtensorMap a_map;   // maps_large viewed {64, M heads, K / 64 chunks} bf16, box {64, 128, 1}
+  CUtensorMap b_map;   // maps_small viewed {64, N heads, K / 64 chunks} bf16, box {64, BN, 1}
   int M, N, BN;
   int64_t K, k_per_split;
   float* C;
@@ -208,7 +213,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gram_tc_kernel(const __grid_con
         if (st >= kGtStages)
           tc::wait_bar(EMPTY(b), ((st / kGtStages) - 1) & 1, abort_flag, p.status);
         tc::mbar_expect_tx(FULL(b), bytes);
-        tc::tma_load_2d(sbase + b * stage + off, map, (int)(k0 + (int64_t)st * 64), y, FULL(b));
+        tc::tma_load_3d(sbase + b * stage + off, map, 0, y, (int)(k0 / 64 + st), FULL(b));
       }
       for (int st = max(0, nsteps - kGtStages); st < nsteps; ++st)
         tc::drain_bar(FULL(st % kGtStages), (st / kGtStages) & 1);
@@ -494,10 +499,11 @@ int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream) {
     gp.K = K;
     gp.C = craw;
     gp.status = a.status;
-    int rc2 = encode_tmap_2d_bf16(&gp.a_map, maps_large, (uint64_t)K, (uint64_t)NL,
-                                  (uint64_t)K * 2, 64, 128);
-    if (!rc2) rc2 = encode_tmap_2d_bf16(&gp.b_map, maps_small, (uint64_t)K, (uint64_t)NS,
-                                        (uint64_t)K * 2, 64, (uint32_t)gp.BN);
+    // chunk-major maps: {64 elements, heads, K / 64 chunks}; heads past N read as zeros
+    int rc2 = encode_tmap_3d_bf16(&gp.a_map, maps_large, 64, (uint64_t)NL, (uint64_t)(K / 64),
+                                  128, (uint64_t)NL * 128, 64, 128, 1);
+    if (!rc2) rc2 = encode_tmap_3d_bf16(&gp.b_map, maps_small, 64, (uint64_t)NS, (uint64_t)(K / 64),
+                                        128, (uint64_t)NS * 128, 64, (uint32_t)gp.BN, 1);
     if (rc2) return rc2;
     const int tm = (NL + 127) / 128, tn = (NS + gp.BN - 1) / gp.BN;
     DeviceContext* ctx = device_context();

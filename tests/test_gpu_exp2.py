@@ -27,8 +27,9 @@ def test_exp2_fma_against_exact_and_mufu():
     # ex2.approx.ftz flushes results below 2^-126; compare where both are normal
     normal = inside & (x > -125.0)
     assert np.max(np.abs(yf[normal] / ym[normal] - 1.0)) < 6e-7
-    # below the clamp the FMA form returns 2^-126 (never a wrapped exponent)
-    assert np.all(yf[~inside] == 2.0 ** -126)
+    # below the clamp the FMA form returns 2^-126 within the polynomial's error (never a
+    # wrapped exponent)
+    assert np.allclose(yf[~inside], 2.0 ** -126, rtol=3e-7, atol=0)
     assert np.all(np.isfinite(yf)) and np.all(yf > 0)
 
 
