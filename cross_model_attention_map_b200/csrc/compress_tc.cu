@@ -103,6 +103,7 @@ struct ExtractParams {
   int dense;
   int64_t dense_tiles;
   int dense_heads;
+  CUtensorMap dense_map;   // dense mode: vals viewed {64, dense_heads, dense_tiles * 64}, box {64, 1, 32}
   float* norm2;
   float* sum1;
   // sender output (extract_tc_kernel<D, true>): V_s bf16 viewed {64, n_k, H_s * d_vs / 64}, box
@@ -750,6 +751,10 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
         tc::tmem_ld_wait();
         if (OUT && c >= 2)   // the P.V MMA of this buffer's previous block has read it
           tc::wait_bar(bar_addr(bars, XP_FREE + 2 * G + sb), ((c >> 1) - 1) & 1, abort_flag, p.status);
+        if (!OUT && p.dense) {   // the tensor store of this warp's previous tile has read it
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          __syncwarp();
+        }
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[16];
@@ -801,6 +806,21 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
         if (lane == 0) tc::mbar_arrive(bar_addr(bars, XP_READY + 2 * G + sb));
       }
       if (base < 0) continue;
+      if (!OUT && p.dense) {
+        // dense mode: the staged 32 rows are one box of the chunk-major maps (32 chunks of head
+        // rank, staged with the same 128-byte swizzle); one tensor store, read asynchronously
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int chunk0 = (int)(base / k) * 64 + (il - lane);
+          asm volatile(
+              "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];\n\t"
+              "cp.async.bulk.commit_group;" ::"l"(&p.dense_map),
+              "r"(0), "r"(rank), "r"(chunk0), "r"(smem_u32(stg))
+              : "memory");
+        }
+        continue;
+      }
       // write 4 tile rows of 128 B per step
       __syncwarp();
       if (base + k <= p.capacity) {
@@ -818,6 +838,7 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
       }
       __syncwarp();
     }
+    if (!OUT && p.dense && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     if (cap_flag && lane == 0) raise_status(p.status, IAMAP_DEV_CAPACITY);
     if (p.norm2) {
 #pragma unroll
@@ -943,6 +964,13 @@ int compress_extract_tc_launch(const CompressArgs& a, cudaStream_t stream) {
   p.dense = a.dense;
   p.dense_tiles = a.dense_tiles;
   p.dense_heads = a.dense && a.dense_tiles > 0 ? (int)(a.capacity / a.dense_tiles) : 0;
+  if (a.dense) {
+    // one warp's 32 rows of a tile: 32 chunks of one head, 128 B each, dense_heads lines apart
+    rc = encode_tmap_3d_bf16(&p.dense_map, a.vals, 64, (uint64_t)p.dense_heads,
+                             (uint64_t)a.dense_tiles * 64, 128, (uint64_t)p.dense_heads * 128, 64,
+                             1, 32);
+    if (rc) return rc;
+  }
   p.norm2 = a.norm2;
   p.sum1 = a.sum1;
   p.tab = a.tab;
