@@ -9,7 +9,7 @@
 //    flattened map of a head is its tiles' rows in order: 64-element chunks c = tile * 64 + row.
 //    The maps of all heads are stored chunk-major (chunk c of head hh is the 128-byte line
 //    c * heads + hh), so that the Gram reads each chunk of 128 heads as one contiguous 16 KB run.
-//    The squared norm and the sum of the bf16 map are accumulated alongside. (Prompts of 2048+
+//    The squared norm and the sum of the bf16 map are accumulated alongside. (Prompts of 1024+
 //    tokens take the tcgen05 compress kernels instead, which write the same layout.)
 // 2. gram_tc_kernel: C_raw = A_large . A_small^T over the flattened maps on the tcgen05 tensor
 //    cores (split-K; operands by TMA with 128-byte swizzle from the chunk-major maps viewed
@@ -439,10 +439,10 @@ int head_match_impl(const HeadMatchArgs& a, cudaStream_t stream) {
   const int NS = a.L_s * a.H_small, NL = a.L_l * a.H_large;
   IAMAP_CUDA_CHECK(cudaMemsetAsync(norms, 0, l.norms + l.craw, stream));
 
-  // Maps on the tensor cores for prompts of 2048+ tokens. At n_used = 1024 (16 row blocks) both
-  // forms took the same time on a B200 (1.12 vs 1.14 ms per calibration): a CTA of the
-  // tensor-core kernels then has at most 8 key tiles to amortise its set-up over.
-  const bool tc_maps = a.n_used >= 2048 && compress_tc_supported(a.d_small, l.nb) &&
+  // Maps on the tensor cores (the tcgen05 compress kernels) for prompts of 1024+ tokens: at
+  // n_used = 1024 a calibration took 0.975 ms this way and 1.037 ms with the mma.sync kernel on
+  // a B200. Shorter prompts keep the mma.sync kernel, whose CTAs need no TMEM set-up.
+  const bool tc_maps = a.n_used >= 1024 && compress_tc_supported(a.d_small, l.nb) &&
                        compress_tc_supported(a.d_large, l.nb);
   if (tc_maps) {
     char* p = ws + l.maps_small + l.maps_large + l.norms + l.craw;

@@ -145,7 +145,7 @@ def test_head_match_small_parity(C, n, n_used, d_small, d_large):
 
 @pytest.mark.parametrize("metric", ["cosine", "pearson"])
 def test_head_match_long_prompt_tensor_core_maps(C, metric):
-    """n_used >= 2048 builds the maps with the tensor-core compress kernels (row statistics, then
+    """n_used >= 1024 builds the maps with the tensor-core compress kernels (row statistics, then
     dense head-major tiles with their sums and norms)."""
     hm = make_head_match(n=2304, L_s=2, H_small=3, d_small=64, L_l=1, H_large=4,
                          d_large=128, noise=0.3, seed=38)
