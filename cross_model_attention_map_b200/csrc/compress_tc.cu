@@ -849,7 +849,9 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
           const int row = 4 * step + (lane >> 3);          // warp-local row
           const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 128 + ((cl ^ (row & 7)) << 4));
           const int tr = (il - lane) + row;                 // tile row of that warp-local row
-          *reinterpret_cast<uint4*>(blk + (int64_t)tr * k * 64 + cl * 8) = val;
+          // streaming store: each tile is read once, by mapped_av, long after this kernel; it
+          // should not displace the keys the grid order keeps in L2
+          __stcs(reinterpret_cast<uint4*>(blk + (int64_t)tr * k * 64 + cl * 8), val);
         }
       } else {
         cap_flag = true;
