@@ -332,8 +332,8 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
         tc::mbar_expect_tx(bar_addr(bars, Q_FULL), kQBytes);
 #pragma unroll
         for (int qp = 0; qp < NPAN; ++qp)
-          tc::tma_load_3d(sQ + qp * kPanel128, &p.q_map, 0, qtok0 + kRows * P, h * NPAN + qp,
-                          bar_addr(bars, Q_FULL));
+          tc::tma_load_3d_hint(sQ + qp * kPanel128, &p.q_map, 0, qtok0 + kRows * P, h * NPAN + qp,
+                               bar_addr(bars, Q_FULL), tc::policy_evict_first());
       }
       tc::prefetch_tmap(&p.k_map);
       for (int T = 0; T < nT; ++T) {
@@ -341,8 +341,10 @@ __global__ void __launch_bounds__(kSThreads, 1) stats_tc_kernel(const __grid_con
         if (T >= kSStages)
           tc::wait_bar(bar_addr(bars, K_EMPTY + st), ((T / kSStages) - 1) & 1, abort_flag, p.status);
         tc::mbar_expect_tx(bar_addr(bars, K_FULL + st), kPanel128);
-        tc::tma_load_3d(sK + st * kKStage + pan * kPanel128, &p.k_map, 0, ktok0 + 128 * T,
-                        h * NPAN + pan, bar_addr(bars, K_FULL + st));
+        // keys are read again by the other row-block pairs of this head group (kept in L2);
+        // the CTA's Q rows are read once
+        tc::tma_load_3d_hint(sK + st * kKStage + pan * kPanel128, &p.k_map, 0, ktok0 + 128 * T,
+                             h * NPAN + pan, bar_addr(bars, K_FULL + st), tc::policy_evict_last());
       }
       for (int T = max(0, nT - kSStages); T < nT; ++T)
         tc::drain_bar(bar_addr(bars, K_FULL + T % kSStages), (T / kSStages) & 1);
@@ -655,8 +657,8 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
       tc::mbar_expect_tx(bar_addr(bars, XQ_FULL), kQBytes);
 #pragma unroll
       for (int pan = 0; pan < NPAN; ++pan)
-        tc::tma_load_3d(sQ + pan * kPanel128, &p.q_map, 0, qtok0 + kRows * P, h * NPAN + pan,
-                        bar_addr(bars, XQ_FULL));
+        tc::tma_load_3d_hint(sQ + pan * kPanel128, &p.q_map, 0, qtok0 + kRows * P, h * NPAN + pan,
+                             bar_addr(bars, XQ_FULL), tc::policy_evict_first());
       for (int t = 0; t < nU; ++t) {
         const int st = t % kXStages;
         if (t >= kXStages)
@@ -665,8 +667,8 @@ __global__ void __launch_bounds__(kThreads, OUT ? 1 : 2) extract_tc_kernel(const
         const int J = ulist[t];
 #pragma unroll
         for (int pan = 0; pan < NPAN; ++pan)
-          tc::tma_load_3d(sK + st * kKStage + pan * kPanel64, &p.k_map, 0, ktok0 + 64 * J,
-                          h * NPAN + pan, bar_addr(bars, XK_FULL + st));
+          tc::tma_load_3d_hint(sK + st * kKStage + pan * kPanel64, &p.k_map, 0, ktok0 + 64 * J,
+                               h * NPAN + pan, bar_addr(bars, XK_FULL + st), tc::policy_evict_last());
         if (OUT) {
           // value tile of block t (both 64-dim halves in one box); its slot is free once the
           // P.V MMA of block t - kVStages completed
