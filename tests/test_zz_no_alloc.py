@@ -5,14 +5,16 @@ reserved nearly all GPU memory for its KV cache at start-up, or one that forbids
 its decode loop because it synchronises the device. For them the library keeps the decode
 kernel's partial sums in a fixed device array instead of a caller workspace. This test calls that
 entry point through the C ABI twice in a row (different inputs, so stale contents of the shared
-array would show) and checks each result against iamap_mapped_av_paged with a workspace, within
-the output tolerance of the other parity tests. The file is named to be collected last.
+array would show) and checks each result against the float64 oracle of the paged decode and against
+iamap_mapped_av_paged with a workspace, within the output tolerance of the other parity tests. The
+file is named to be collected last.
 """
 
 import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from synth import make_decode
 
 from _gpu_common import bf16, check_output
@@ -44,7 +46,7 @@ def _no_alloc(C, dw, p, W, vp, pt, cl):
     return out
 
 
-def test_no_alloc_decode_matches_workspace_entry_point():
+def test_no_alloc_decode_matches_oracle_and_workspace_entry_point():
     from cross_model_attention_map_b200 import iamap as C
     cases = [make_decode(seed=41),                                     # batch 4, context 8704
              make_decode(batch=3, ctx=500, H_s=5, H_r=16, d_v=128, page_size=16,
@@ -54,6 +56,7 @@ def test_no_alloc_decode_matches_workspace_entry_point():
         got = _no_alloc(C, dw, *args)
         ref = _with_workspace(C, dw, *args)
         torch.cuda.synchronize()
+        check_output(got.cpu().numpy(), O.mapped_av_paged(dw), "no-alloc decode vs oracle")
         check_output(got.cpu().numpy(), ref.cpu().numpy().astype(np.float64), "no-alloc decode")
 
 
