@@ -104,6 +104,8 @@ def test_tiny_config_full_parity(C):
     ([640], 3, 2, 128, 1.0, (0, 0.0)),                    # keep everything
     ([450, 70], 7, 9, 64, 0.3, (16, 2.0)),                # aggressive sparsity
     ([130, 0, 64, 0], 4, 4, 64, 0.9, (0, 0.0)),           # empty sequences inside the batch
+    ([600, 77], 64, 32, 128, 0.9, (0, 0.0)),              # the largest head counts: every head-mask
+                                                          # bit, 32 receivers in clusters of 8
 ])
 def test_varlen_parity(C, seqlens, H_s, H_r, d, tau, bias):
     wl = make_prefill(seqlens, H_s=H_s, d=d, H_r=H_r, d_v=d, B=64, tau=tau, std=1.5, sink=True,
