@@ -15,9 +15,9 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("seqlens,H_s,H_r,H_kv,d,tau,bias", [
-    ([300, 70, 1], 5, 6, 6, 64, 0.9, (0, 0.0)),        # tensor-core mapped_av
+    ([300, 70, 1], 5, 14, 14, 64, 0.9, (0, 0.0)),      # tensor-core mapped_av (4-CTA clusters)
     ([260, 90], 4, 40, 8, 64, 0.9, (0, 0.0)),          # H_r > 32: the CUDA-core mapped_av
-    ([500], 6, 8, 8, 128, 0.95, (128, 2.0)),           # d = 128, local bias
+    ([500], 6, 8, 8, 128, 0.95, (128, 2.0)),           # d = 128, local bias, CUDA-core mapped_av
 ])
 def test_layers_in_one_launch(seqlens, H_s, H_r, H_kv, d, tau, bias):
     from cross_model_attention_map_b200 import iamap as C

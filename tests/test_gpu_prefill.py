@@ -114,7 +114,9 @@ def test_varlen_parity(C, seqlens, H_s, H_r, d, tau, bias):
 
 
 @pytest.mark.parametrize("seqlens,H_s,H_r,H_kv,d", [
-    ([300, 90], 6, 8, 2, 64),      # tensor-core cluster kernel, 4 receivers per value head
+    ([300, 90], 20, 8, 2, 64),     # tensor-core cluster kernel (2 CTAs, H_s > 16), 4 receivers
+                                   # per value head
+    ([300, 90], 6, 8, 2, 64),      # the CUDA-core kernel (2-CTA cluster, few sender heads)
     ([200], 5, 12, 3, 128),        # tensor-core, groups across CTA boundaries
     ([260, 40], 4, 40, 8, 64),     # H_r > 32: the CUDA-core kernel
 ])
