@@ -14,7 +14,7 @@
 //     whose lines are the K-stack of an MN-major, 128-byte-swizzled operand. It mixes them for ALL receiver
 //     heads: D[128 positions][N = H_r] = P[128][K = heads] . W'[N][K] with tcgen05.mma, where W'
 //     holds the W columns of the present heads (zero past them).
-//   * The mixed rows are rounded to bf16, transposed through a 2 KB per-warp scratch into 16-byte
+//   * The mixed rows are rounded to bf16, transposed (stmatrix) through a 2 KB per-warp scratch into 16-byte
 //     runs of 8 positions of one receiver head, and stored with st.async straight into the receive
 //     buffer of the CTA owning that head, at their place in its K-major, 128-byte-swizzled tile;
 //     the bytes count on that CTA's mbarrier.
@@ -397,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
     const uint32_t lane_base = (uint32_t)(32 * e) << 16;
     const int ew = eg * 4 + (warp - (eg ? 13 : 2));   // 0..7
     unsigned char* scr = smem + p.off_scr + ew * 2048;   // [32 heads][32 positions] bf16
+    const uint32_t scr_u32 = smem_u32(scr);
     const int o = lane & 3;               // this lane's 16-byte run: positions 8*o .. 8*o+7
     const int rq = lane >> 2;             // this lane's heads: 8*v + rq
     const int nch = c1 - c0;
@@ -420,16 +421,24 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         if (releaser)
           for (int jj = 0; jj < nj; ++jj) tc::mbar_arrive(bar_addr(bars, P_EMPTY + (q + cc + jj) % NP));
         tc::tc_fence_after();
+        // chunk j in the fragment shape: v[j][16 hh + 4 m + k] = position 16 hh + 8 (k >= 2) + lane / 4
+        // of this warp's 32, receiver head 8 m + 2 (lane % 4) + (k & 1)
         uint32_t v[2][32];
         const uint32_t ta = tmem + lane_base + (uint32_t)kMixCol + (uint32_t)(2 * gs) * (uint32_t)p.NR;
         if (p.NR == 32) {
-          IAMAP_TMEM_LD32(ta, v[0]);
-          if (nj == 2) IAMAP_TMEM_LD32(ta + 32u, v[1]);
+          IAMAP_TMEM_LD_FRAG16(ta, v[0]);
+          IAMAP_TMEM_LD_FRAG16(ta + (16u << 16), v[0] + 16);
+          if (nj == 2) {
+            IAMAP_TMEM_LD_FRAG16(ta + 32u, v[1]);
+            IAMAP_TMEM_LD_FRAG16(ta + 32u + (16u << 16), v[1] + 16);
+          }
         } else {
-          IAMAP_TMEM_LD16(ta, v[0]);
-          if (nj == 2) IAMAP_TMEM_LD16(ta + 16u, v[1]);
-#pragma unroll
-          for (int i = 16; i < 32; ++i) v[0][i] = v[1][i] = 0u;
+          IAMAP_TMEM_LD_FRAG8(ta, v[0]);
+          IAMAP_TMEM_LD_FRAG8(ta + (16u << 16), v[0] + 16);
+          if (nj == 2) {
+            IAMAP_TMEM_LD_FRAG8(ta + 16u, v[1]);
+            IAMAP_TMEM_LD_FRAG8(ta + 16u + (16u << 16), v[1] + 16);
+          }
         }
         tc::tmem_ld_wait();
         tc::tc_fence_before();
@@ -440,11 +449,24 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         for (int j = 0; j < 2; ++j) {
           if (j >= nj) break;
           const int ch = c0 + cc + j;
-          // transpose: position = lane, head = register  ->  16-byte runs of one head
+          // transpose into [head][32 positions] rows: each 8 positions x 8 heads tile is stored
+          // transposed by stmatrix, so that a row holds 16-byte runs of one head; the run of
+          // position octet po of head r sits at 16 * (po ^ ((r >> 1) & 3)), which keeps both
+          // the stores and the reads below free of bank conflicts
 #pragma unroll
-          for (int r = 0; r < 32; ++r)
-            if (r < p.NR)
-              reinterpret_cast<__nv_bfloat16*>(scr)[r * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[j][r]));
+          for (int po = 0; po < 4; ++po) {
+            const int b = 16 * (po >> 1) + 2 * (po & 1);
+            const uint32_t a = scr_u32 + (uint32_t)lane * 64u + ((uint32_t)(po ^ ((lane >> 1) & 3)) << 4);
+            const uint32_t q0 = pack_bf16(__uint_as_float(v[j][b]), __uint_as_float(v[j][b + 1]));
+            const uint32_t q1 = pack_bf16(__uint_as_float(v[j][b + 4]), __uint_as_float(v[j][b + 5]));
+            if (p.NR == 32) {
+              const uint32_t q2 = pack_bf16(__uint_as_float(v[j][b + 8]), __uint_as_float(v[j][b + 9]));
+              const uint32_t q3 = pack_bf16(__uint_as_float(v[j][b + 12]), __uint_as_float(v[j][b + 13]));
+              tc::stmatrix_x4_trans(a, q0, q1, q2, q3);
+            } else {
+              tc::stmatrix_x4_trans(a, q0, q1, 0u, 0u);   // heads 16-31 do not exist
+            }
+          }
           __syncwarp();
           const int pos0 = 32 * e;                          // this warp's first position in the chunk
           const int arow = 2 * ch + (pos0 >> 6);            // tile row
@@ -454,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
           for (int vv = 0; vv < 4; ++vv) {
             const int r = 8 * vv + rq;
             if (r < p.H_r) {
-              const uint4 val = *reinterpret_cast<const uint4*>(scr + r * 64 + o * 16);
+              const uint4 val = *reinterpret_cast<const uint4*>(scr + r * 64 + ((o ^ ((r >> 1) & 3)) << 4));
               const uint32_t c2 = (uint32_t)(r >> 2);
               const uint32_t dst = tc::map_to_cta(recv_local + (uint32_t)(r & 3) * 8192u + row_off, c2);
               tc::st_async_v4(dst, val, tc::map_to_cta(rbar_local, c2));

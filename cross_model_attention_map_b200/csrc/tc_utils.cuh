@@ -251,6 +251,35 @@ __device__ __forceinline__ void mma_commit_to_cluster(uint32_t bar, uint16_t cta
         "=r"(v[31])                                                                             \
       : "r"(taddr))
 
+// 16 TMEM lanes x 32 columns in the fragment shape (16x256b, 4 repetitions): register 4m + k of
+// thread t holds lane (k >= 2 ? 8 : 0) + t / 4 and column 8m + 2 (t % 4) + (k & 1) (checked on the
+// B200 with known values), i.e. the row/column-pair layout that stmatrix takes.
+#define IAMAP_TMEM_LD_FRAG16(taddr, v)                                                          \
+  asm volatile(                                                                                 \
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"  \
+      "%14,%15}, [%16];"                                                                        \
+      : "=r"((v)[0]), "=r"((v)[1]), "=r"((v)[2]), "=r"((v)[3]), "=r"((v)[4]), "=r"((v)[5]),    \
+        "=r"((v)[6]), "=r"((v)[7]), "=r"((v)[8]), "=r"((v)[9]), "=r"((v)[10]), "=r"((v)[11]),   \
+        "=r"((v)[12]), "=r"((v)[13]), "=r"((v)[14]), "=r"((v)[15])                              \
+      : "r"(taddr))
+
+// The same for 16 columns (2 repetitions, registers 0-7).
+#define IAMAP_TMEM_LD_FRAG8(taddr, v)                                                           \
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"        \
+               : "=r"((v)[0]), "=r"((v)[1]), "=r"((v)[2]), "=r"((v)[3]), "=r"((v)[4]),           \
+                 "=r"((v)[5]), "=r"((v)[6]), "=r"((v)[7])                                        \
+               : "r"(taddr))
+
+// Four 8 x 8 b16 tiles stored transposed: register i of thread t holds row t / 4, columns
+// 2 (t % 4) and 2 (t % 4) + 1 (low half first) of tile i; thread 8i + k gives the address of the
+// 16-byte memory row k of tile i, which receives column k of the tile.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                                  uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+               "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
 #define IAMAP_TMEM_LD16(taddr, v)                                                               \
   asm volatile(                                                                                 \
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"  \
