@@ -125,7 +125,7 @@ constexpr uint32_t kTmemCols = 512;
 enum {
   P_FULL = 0, P_EMPTY = P_FULL + kMaxNP, W_FULL = P_EMPTY + kMaxNP, W_EMPTY = W_FULL + 2,
   D_FULL = W_EMPTY + 2, D_EMPTY = D_FULL + kNG, RECV_FULL = D_EMPTY + kNG, BUF_FREE = RECV_FULL + kRecv,
-  V_FULL = BUF_FREE + kRecv, PV_DONE = V_FULL + kNV, O_FULL = PV_DONE + 2, MIX_DONE = O_FULL + 1,
+  V_FULL = BUF_FREE + kRecv, O_FULL = V_FULL + kNV, MIX_DONE = O_FULL + 1,
   NUM_BARS = MIX_DONE + 1
 };
 
@@ -297,8 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
     }
   } else if (warp == 6 || warp == 11 || warp == 17 || warp == 18) {
     // ------------------------------ V tiles (one warp per receiver head) ----------------------
-    // slot rl holds V_rl[J] of the current block; it is refilled once this CTA's P.V of the
-    // previous block has completed (PV_DONE), so each slot is used once per block
+    // slot rl holds V_rl[J] of the current block; it is refilled once the P.V of the previous
+    // block has completed in every CTA of the cluster (the receive-buffer release of that round,
+    // which includes this CTA's own), so each slot is used once per block. That barrier cannot
+    // run two phases ahead of this wait: its next phase needs this CTA's P.V of block t, which
+    // needs the V tiles loaded after it.
     const int vw = warp == 6 ? 0 : warp == 11 ? 1 : warp == 17 ? 2 : 3;
     const int halves = p.d_v / 64;
     if (lane == 0) {
@@ -308,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
       for (int t = 0; t < T; ++t) {
         const int J = J_next;
         if (t + 1 < T) J_next = p.col_idx[u0 + t + 1];
-        if (t >= 1) tc::wait_bar(bar_addr(bars, PV_DONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, abort_flag, p.status);
+        if (t >= 1) tc::wait_bar(bar_addr(bars, BUF_FREE + (t - 1) % kRecv), ((t - 1) / kRecv) & 1, abort_flag, p.status);
         for (int rl = vw; rl < G; rl += kVWarps) {
           tc::mbar_expect_tx(bar_addr(bars, V_FULL + rl), v_stage);
           tc::tma_load_3d_hint(sbase + p.off_v + rl * v_stage, &p.v_map, 0, seq0 + J * 64,
@@ -353,8 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
           }
           tc::mma_commit(bar_addr(bars, D_FULL + gs));
         }
-        q += nch;
-        tc::mma_commit(bar_addr(bars, W_EMPTY + ws));
+        q += nch;   // W' of this block is released by the readout of its last pair
       }
       tc::mma_commit(bar_addr(bars, MIX_DONE));
       tc::drain_bar(bar_addr(bars, MIX_DONE), 0);   // every mixing MMA completed before TMEM is freed
@@ -383,7 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
             tc::mma_bf16(tmem + (uint32_t)rl * 64u, a, b, id_pv, (t > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        tc::mma_commit(bar_addr(bars, PV_DONE + (t & 1)));
         tc::mma_commit_to_cluster(bar_addr(bars, BUF_FREE + rs), all_ctas);
       }
       tc::mma_commit(bar_addr(bars, O_FULL));
@@ -417,9 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1) mapped_av_tc_kernel(const __grid_
         const int gs = eg * kNGh + gp % kNGh;
         const int nj = min(2, nch - cc);
         tc::wait_bar(bar_addr(bars, D_FULL + gs), (gp / kNGh) & 1, abort_flag, p.status);
-        // the pair's mixing MMAs completed: their sender slots can be refilled
-        if (releaser)
+        // the pair's mixing MMAs completed: their sender slots can be refilled, and after the
+        // block's last pair (its commit covers every earlier MMA) the block's W' as well
+        if (releaser) {
           for (int jj = 0; jj < nj; ++jj) tc::mbar_arrive(bar_addr(bars, P_EMPTY + (q + cc + jj) % NP));
+          if (cc + 2 >= nch) tc::mbar_arrive(bar_addr(bars, W_EMPTY + (t & 1)));
+        }
         tc::tc_fence_after();
         // chunk j in the fragment shape: v[j][16 hh + 4 m + k] = position 16 hh + 8 (k >= 2) + lane / 4
         // of this warp's 32, receiver head 8 m + 2 (lane % 4) + (k & 1)
