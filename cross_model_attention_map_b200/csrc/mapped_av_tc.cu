@@ -99,7 +99,7 @@ namespace tcav {
 
 constexpr int kG = 4;            // receiver heads per CTA (O in TMEM: 4 x 64 columns)
 constexpr int kMaxNP = 12;       // sender-slice ring: as many slots as shared memory allows
-// A thread that issues TMA loads waits ~5 ns per 128-byte line of the box (measured on this B200:
+// A thread that issues TMA loads waits ~5 ns per 128-byte line of the box (measured on a B200:
 // 0.31 us for a 16 KB contiguous box, 0.49 us for a V tile spread over 64 tokens, i.e. 33-52 GB/s
 // per issuing thread, against ~130 GB/s per SM from L2 with four issuers), so the loads are
 // spread over several producer warps: four for the sender slices and one per receiver head for
@@ -110,7 +110,7 @@ constexpr int kMaxNP = 12;       // sender-slice ring: as many slots as shared m
 constexpr int kPWarps = 4, kVWarps = 4;
 constexpr int kND = 8;           // mixing-result TMEM slots (chunks)
 constexpr int kNG = kND / 2;     // ... committed and released in pairs of chunks (one commit costs
-                                 // ~90 ns of issue time on this B200, an MMA ~25 ns)
+                                 // ~90 ns of issue time on a B200, an MMA ~25 ns)
 constexpr int kNGh = kNG / 2;    // pair slots of each readout group: even pairs of a block use
                                  // slots 0-1, odd pairs slots 2-3, so that every slot has one
                                  // consumer that takes its phases in order
