@@ -12,8 +12,10 @@
 //   3. warp w computes O_r[16 rows] += P_r . V_r[J] with mma.sync (bf16 in, fp32 accumulate)
 //      for receiver head r = w / 4 of the group, V_r[J] staged in shared memory.
 // The output rows are written once, after the last column block.
-// This form serves receiver layers wider than the tensor-core kernel's cluster (H_r > 32); the
-// tensor-core, cluster-cooperative kernel (mapped_av_tc.cu) handles H_r <= 32.
+// This form serves receiver layers wider than the tensor-core kernel's cluster (H_r > 32) and
+// narrow ones whose cluster would have one CTA, or two with at most 16 sender heads (there it is
+// the faster of the two; see use_tensor_core_path below); the tensor-core, cluster-cooperative
+// kernel (mapped_av_tc.cu) handles the rest of H_r <= 32.
 #include "internal.h"
 
 namespace iamap {
